@@ -1,0 +1,328 @@
+"""Pins for the CPU oracle: facts fixed by the pages and by mathematics,
+independent of the oracle's own code.
+
+Each pin returns normally when it holds and raises ``AssertionError`` when it
+does not. ``run_pins(oracle)`` runs them all and returns the failures, so the
+same pins can be run against the real oracle (no failure allowed) and against
+copies of it with a planted mistake (at least one failure required).
+
+What pins what:
+* the hand-worked examples in ``tests/golden`` (exact rational values
+  derived from the FBI-linear paragraph and BitNet Eq.(1)-(8));
+* closed forms: all-ones input gives alpha_j*(#pos - #neg); an all-positive
+  row gives alpha * (exact sum of x); alternating +-1 input quantises to
+  +-127;
+* the W1A1 identity dot = K - 2*popcount(a XOR b), brute-forced over every
+  pair of sign vectors for small K, and the W1A16 forward fed +-1 inputs;
+* independent library routines: ``numpy.packbits`` for the packed layout,
+  ``math.fsum`` (exact sums) for the scales;
+* invariants: negation, scaling by powers of two, integer shifts, constant
+  tokens, exact .5 ties (round half to even).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _frac(s) -> Fraction:
+    return Fraction(s)
+
+
+def _bf16_bits_of(values) -> np.ndarray:
+    """bf16 patterns of values that are exactly representable in bf16."""
+    f = np.asarray([float(v) for v in values], dtype=np.float32)
+    u = f.view(np.uint32)
+    assert np.all((u & 0xFFFF) == 0), "value not exact in bf16"
+    return (u >> 16).astype(np.uint16)
+
+
+def _bf16_values(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _to_bf16_bits(f32: np.ndarray) -> np.ndarray:
+    """Round fp32 to bf16 (nearest even) -- input generation only."""
+    u = np.ascontiguousarray(f32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return r.astype(np.uint16)
+
+
+def _popcounts(words: np.ndarray) -> np.ndarray:
+    """Set bits per row of a uint32 array (rows = leading axis)."""
+    return np.array([sum(int(w).bit_count() for w in row) for row in words], dtype=np.int64)
+
+
+def _packbits_rows(bits: np.ndarray, K: int) -> np.ndarray:
+    """Independent statement of the packed layout through numpy.packbits:
+    little bit order inside each byte, little-endian bytes inside each word."""
+    N = bits.shape[0]
+    words = (K + 31) // 32
+    padded = np.zeros((N, words * 32), dtype=np.uint8)
+    padded[:, :K] = bits
+    by = np.packbits(padded, axis=1, bitorder="little")
+    return by.view("<u4").reshape(N, words).astype(np.uint32)
+
+
+# ---------------------------------------------------------------- examples
+
+
+def pin_example_a_pack(o):
+    ex = _load("fbi_example_a.json")
+    W = np.array([[float(_frac(v)) for v in row] for row in ex["W"]], dtype=np.float32)
+    packed, alpha = o.pack_fbi(W)
+    assert packed[:, 0].tolist() == ex["packed"], packed[:, 0].tolist()
+    assert [Fraction(float(a)) for a in alpha] == [_frac(a) for a in ex["alpha"]], alpha
+    u = ex["unbalanced_row"]
+    Wu = np.array([[float(_frac(v)) for v in u["W"]]], dtype=np.float32)
+    pu, au = o.pack_fbi(Wu)
+    assert int(pu[0, 0]) == u["packed"] and Fraction(float(au[0])) == _frac(u["alpha"])
+    y = o.w1a16(_bf16_bits_of([1, 1, 1, 1])[None, :], pu, au, 4)
+    assert Fraction(float(y[0, 0])) == _frac(u["y_all_ones"]), y
+
+
+def pin_example_a_forward(o):
+    ex = _load("fbi_example_a.json")
+    packed = np.array(ex["packed"], dtype=np.uint32)[:, None]
+    alpha = np.array([float(_frac(a)) for a in ex["alpha"]], dtype=np.float32)
+    for case in ex["cases"]:
+        x = _bf16_bits_of([_frac(v) for v in case["x"]])[None, :]
+        y = o.w1a16(x, packed, alpha, ex["K"])
+        assert [Fraction(float(v)) for v in y[0]] == [_frac(v) for v in case["y"]], y
+
+
+def pin_example_b_pack(o):
+    ex = _load("bitnet_example_b.json")
+    W = np.array([[float(_frac(v)) for v in row] for row in ex["W"]], dtype=np.float32)
+    packed, alpha, beta = o.pack_bitnet(W)
+    assert packed[:, 0].tolist() == ex["packed"], packed[:, 0].tolist()
+    assert Fraction(alpha) == _frac(ex["alpha"]), alpha
+    assert Fraction(beta) == _frac(ex["beta"]), beta
+
+
+def pin_example_b_forward(o):
+    ex = _load("bitnet_example_b.json")
+    packed = np.array(ex["packed"], dtype=np.uint32)[:, None]
+    beta = float(_frac(ex["beta"]))
+    for tok in ex["tokens"]:
+        x = _bf16_bits_of([_frac(v) for v in tok["x"]])[None, :]
+        xq, gamma, pre = o.ln_absmax_quant(x, ex["eps"], want_pre=True)
+        assert xq[0].tolist() == tok["xq"], xq
+        # pre-round values: exact up to fp64 rounding of the LN steps
+        for got, want in zip(pre[0], tok["pre"]):
+            assert abs(got - float(_frac(want))) <= 1e-12 * 128, (pre, tok["pre"])
+        assert abs(gamma[0] - float(tok["gamma"])) <= 4e-16 * float(tok["gamma"]), gamma
+        acc = o.w1a8_acc(xq, packed, ex["K"])
+        assert acc[0].tolist() == tok["acc"], acc
+        y = o.w1a8_rescale(acc, gamma, beta)
+        for got, want in zip(y[0], tok["y"]):
+            assert abs(got - float(want)) <= 1e-15 * abs(float(want)), (y, tok["y"])
+
+
+def pin_round_half_even_ties(o):
+    ex = _load("rne_tie.json")
+    c = ex["magnitudes"]
+    x = _bf16_bits_of(list(c) + [-v for v in c])[None, :]
+    xq, gamma = o.ln_absmax_quant(x, ex["eps"])
+    want = list(ex["xq_magnitudes"]) + [-v for v in ex["xq_magnitudes"]]
+    assert xq[0].tolist() == want, xq[0].tolist()
+    assert Fraction(float(gamma[0])) == _frac(ex["gamma"]), gamma
+
+
+# ------------------------------------------------------------ closed forms
+
+
+def _random_case(seed, N, K, M=3, mean=0.0):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((N, K)) * 0.02 + mean).astype(np.float32)
+    x = _to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    return W, x
+
+
+def pin_packed_layout_numpy(o):
+    for K in (32, 96, 100, 7):
+        W, _ = _random_case(11 + K, 9, K)
+        W[0, : min(K, 5)] = 0.0  # zeros must pack as -1 (bit clear)
+        packed, _ = o.pack_fbi(W)
+        assert np.array_equal(packed, _packbits_rows((W > 0).astype(np.uint8), K)), K
+
+
+def pin_fbi_alpha_exact_sum(o):
+    W, _ = _random_case(5, 17, 300)
+    _, alpha = o.pack_fbi(W)
+    for j in range(W.shape[0]):
+        want = np.float32(math.fsum(abs(float(v)) for v in W[j]) / W.shape[1])
+        assert abs(int(alpha[j].view(np.int32)) - int(want.view(np.int32))) <= 1, (j, alpha[j], want)
+
+
+def pin_bitnet_global_scalars(o):
+    W, _ = _random_case(6, 23, 128, mean=0.001)
+    packed, alpha, beta = o.pack_bitnet(W)
+    n = W.size
+    a_exact = math.fsum(float(v) for v in W.ravel()) / n
+    b_exact = math.fsum(abs(float(v)) for v in W.ravel()) / n
+    assert abs(alpha - a_exact) <= 1e-12 * abs(a_exact), (alpha, a_exact)
+    assert abs(beta - b_exact) <= 1e-14 * b_exact, (beta, b_exact)
+    # signs of W - alpha, with the boundary decided on the exact mean
+    bits = (W.astype(np.float64) > a_exact).astype(np.uint8)
+    assert np.array_equal(packed, _packbits_rows(bits, W.shape[1]))
+
+
+def pin_bitnet_sign_at_mean(o):
+    # every weight equal to the global mean maps to -1 ([BitNet] Eq.(2): <= 0 -> -1)
+    W = np.array([[1.0, 2.0, 3.0, 2.0], [2.0, 0.0, 4.0, 2.0]], dtype=np.float32)  # mean 2
+    packed, alpha, _ = o.pack_bitnet(W)
+    assert alpha == 2.0
+    assert packed[:, 0].tolist() == [0b0100, 0b0100], packed[:, 0].tolist()
+
+
+def pin_all_ones_closed_form(o):
+    for K in (64, 130):
+        W, _ = _random_case(21 + K, 13, K)
+        packed, alpha = o.pack_fbi(W)
+        y = o.w1a16(_bf16_bits_of([1] * K)[None, :], packed, alpha, K)
+        pos = _popcounts(packed)
+        want = alpha.astype(np.float64) * (2 * pos - K)
+        assert np.array_equal(y[0], want), (y[0], want)
+
+
+def pin_all_positive_row_is_plain_sum(o):
+    K = 32
+    rng = np.random.default_rng(3)
+    x = _to_bf16_bits(rng.standard_normal((2, K)).astype(np.float32))
+    W = np.abs(rng.standard_normal((1, K))).astype(np.float32) + 0.5
+    packed, alpha = o.pack_fbi(W)
+    assert int(packed[0, 0]) == 0xFFFFFFFF
+    y = o.w1a16(x, packed, alpha, K)
+    for m in range(2):
+        s = math.fsum(_bf16_values(x[m]).tolist())
+        assert y[m, 0] == float(alpha[0]) * s, (y[m, 0], s)
+
+
+def pin_negation(o):
+    W, x = _random_case(31, 19, 160, M=4)
+    packed, alpha = o.pack_fbi(W)
+    y = o.w1a16(x, packed, alpha, 160)
+    yn = o.w1a16(x ^ np.uint16(0x8000), packed, alpha, 160)
+    assert np.array_equal(yn, -y)
+
+
+def pin_w1a1_identity_bruteforce(o):
+    for K in (1, 2, 3, 5, 6, 10):
+        vals = np.arange(1 << K, dtype=np.uint32)[:, None]
+        dot = o.w1a1(vals, vals, K)
+        xor = vals[:, 0][:, None] ^ vals[:, 0][None, :]
+        pc = np.vectorize(lambda v: int(v).bit_count())(xor)
+        assert np.array_equal(dot, K - 2 * pc), K
+
+
+def pin_w1a1_multiword(o):
+    K = 77
+    rng = np.random.default_rng(8)
+    wpr = (K + 31) // 32
+    a = rng.integers(0, 2**32, size=(5, wpr), dtype=np.uint64).astype(np.uint32)
+    b = rng.integers(0, 2**32, size=(6, wpr), dtype=np.uint64).astype(np.uint32)
+    a[:, -1] &= (1 << (K % 32)) - 1
+    b[:, -1] &= (1 << (K % 32)) - 1
+    dot = o.w1a1(a, b, K)
+    for i in range(5):
+        for j in range(6):
+            pc = sum(int(u ^ v).bit_count() for u, v in zip(a[i], b[j]))
+            assert dot[i, j] == K - 2 * pc
+
+
+def pin_w1a16_on_pm1_inputs_is_w1a1(o):
+    # feeding the W1A16 forward +-1 activations (alpha = 1) must give the W1A1 dot
+    K = 10
+    vals = np.arange(1 << K, dtype=np.uint32)[:, None]
+    bits = ((vals >> np.arange(K, dtype=np.uint32)) & 1).astype(np.int64)
+    x = _bf16_bits_of((2 * bits - 1).ravel()).reshape(1 << K, K)
+    sel = vals[::37]
+    y = o.w1a16(x, sel, np.ones(sel.shape[0], dtype=np.float32), K)
+    dot = o.w1a1(vals, sel, K)
+    assert np.array_equal(y, dot.astype(np.float64))
+
+
+def pin_quant_invariants(o):
+    rng = np.random.default_rng(12)
+    M, K = 6, 96
+    xi = rng.integers(-100, 101, size=(M, K)).astype(np.float32)
+    x = _bf16_bits_of(xi.ravel()).reshape(M, K)
+    xq, gamma = o.ln_absmax_quant(x)
+    # every token's largest |x - mu| sits on the clamp; all codes in range
+    assert np.all(np.abs(xq).max(axis=1) == 127)
+    assert np.all(np.abs(xq.astype(np.int32)) <= 127)
+    # scaling by a power of two leaves the codes unchanged (LN cancels it)
+    xs = _bf16_bits_of((xi * 4).ravel()).reshape(M, K)
+    assert np.array_equal(o.ln_absmax_quant(xs)[0], xq)
+    # shifting every token by an integer leaves the codes unchanged
+    xh = _bf16_bits_of((xi + 64).ravel()).reshape(M, K)
+    assert np.array_equal(o.ln_absmax_quant(xh)[0], xq)
+    # negation negates the codes
+    assert np.array_equal(o.ln_absmax_quant(x ^ np.uint16(0x8000))[0], -xq)
+
+
+def pin_alternating_and_constant_tokens(o):
+    K = 64
+    alt = np.array([1.0 if k % 2 == 0 else -1.0 for k in range(K)], dtype=np.float32)
+    const = np.full(K, 3.0, dtype=np.float32)
+    x = np.stack([_bf16_bits_of(alt), _bf16_bits_of(const)])
+    xq, gamma = o.ln_absmax_quant(x)
+    assert xq[0].tolist() == [127 if k % 2 == 0 else -127 for k in range(K)]
+    assert xq[1].tolist() == [0] * K and gamma[1] == 0.0
+    W, _ = _random_case(41, 11, K)
+    packed, _ = o.pack_fbi(W)
+    acc = o.w1a8_acc(xq, packed, K)
+    signs = 2 * ((packed[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(11, -1)[:, :K].astype(np.int64) - 1
+    alt_sign = np.array([1 if k % 2 == 0 else -1 for k in range(K)], dtype=np.int64)
+    assert np.array_equal(acc[0], 127 * (signs @ alt_sign))
+    assert np.array_equal(acc[1], np.zeros(11, dtype=np.int64))
+    y = o.w1a8_rescale(acc, gamma, 0.25)
+    assert np.all(y[1] == 0.0)
+
+
+def pin_acc_with_unit_codes(o):
+    K = 160
+    W, _ = _random_case(51, 14, K)
+    packed, _ = o.pack_fbi(W)
+    acc = o.w1a8_acc(np.ones((1, K), dtype=np.int8), packed, K)
+    assert np.array_equal(acc[0], 2 * _popcounts(packed) - K)
+
+
+def pin_sampled_equals_full(o):
+    W, x = _random_case(61, 9, 64, M=5)
+    packed, alpha = o.pack_fbi(W)
+    y = o.w1a16(x, packed, alpha, 64)
+    ms = np.array([0, 4, 2, 3], dtype=np.int64)
+    js = np.array([8, 0, 5, 5], dtype=np.int64)
+    assert np.array_equal(o.w1a16_at(x, packed, alpha, 64, ms, js), y[ms, js])
+    xq, _ = o.ln_absmax_quant(x)
+    acc = o.w1a8_acc(xq, packed, 64)
+    assert np.array_equal(o.w1a8_acc_at(xq, packed, 64, ms, js), acc[ms, js])
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]
+
+
+def run_pins(oracle) -> list[tuple[str, str]]:
+    """Run every pin; return [(name, message)] for those that failed."""
+    failures = []
+    for pin in PINS:
+        try:
+            pin(oracle)
+        except AssertionError as e:  # a pin that does not hold
+            failures.append((pin.__name__, str(e)[:200]))
+        except Exception as e:  # a broken oracle may also crash a pin
+            failures.append((pin.__name__, f"{type(e).__name__}: {str(e)[:200]}"))
+    return failures

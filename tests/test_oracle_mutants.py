@@ -1,0 +1,77 @@
+"""The pins catch plausible mistakes in the oracle (no GPU).
+
+Each case plants one mistake in a private copy of ``oracle/oracle.c``,
+compiles it, and requires that at least one pin fails on the broken copy.
+The real oracle source is never modified.
+"""
+import os
+import shutil
+import tempfile
+
+import pytest
+
+import oracle as oracle_pkg
+from oracle import build as oracle_build
+
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle_pkg.__file__), "oracle.c")
+
+# (name, text in the oracle, replacement) -- each a mistake a reader might make
+MUTANTS = [
+    ("sign_of_zero_is_plus", "return v > 0.0 ? 1 : -1;", "return v >= 0.0 ? 1 : -1;"),
+    ("msb_first_bits", "(k % 32)", "(31 - k % 32)"),
+    ("row_stride_floor", "return (K + 31) / 32;", "return K / 32 > 0 ? K / 32 : 1;"),
+    ("fbi_alpha_signed_mean", "abs_sum += fabs(w);", "abs_sum += w;"),
+    ("fbi_alpha_divides_by_n", "alpha[j] = (float)(abs_sum / (double)K);",
+     "alpha[j] = (float)(abs_sum / (double)N);"),
+    ("bitnet_no_shift", "sign_pm1((double)W[j * K + k] - alpha)", "sign_pm1((double)W[j * K + k])"),
+    ("bitnet_beta_from_signed_sum", "*beta_out = abs_sum / count;", "*beta_out = sum / count;"),
+    ("bitnet_alpha_per_row_count", "double alpha = sum / count;", "double alpha = sum / (double)K;"),
+    ("dropped_last_term", "for (int64_t k = 0; k < K; ++k)\n        dot +=",
+     "for (int64_t k = 0; k < K - 1; ++k)\n        dot +="),
+    ("alpha_indexed_by_token", "return (double)alpha[j] * dot;", "return (double)alpha[m] * dot;"),
+    ("sample_index_swapped", "y[i] = w1a16_one(x, packed, alpha, K, ms[i], js[i]);",
+     "y[i] = w1a16_one(x, packed, alpha, K, js[i] % 1, js[i]);"),
+    ("variance_unbiased", "double var = sq / (double)K;", "double var = sq / (double)(K - 1);"),
+    ("eps_outside_sqrt", "double root = sqrt(var + eps);", "double root = sqrt(var) + eps;"),
+    ("no_mean_subtraction",
+     "double ln = (bf16_value(row[k]) - mu) / root;\n            if (fabs(ln) > gamma)",
+     "double ln = bf16_value(row[k]) / root;\n            if (fabs(ln) > gamma)"),
+    ("round_half_away", "double r = nearbyint(v);", "double r = round(v);"),
+    ("truncate_not_round", "double r = nearbyint(v);", "double r = trunc(v);"),
+    ("no_clamp", "if (r > 127.0) r = 127.0;", ""),
+    ("clamp_to_128", "if (r < -127.0) r = -127.0;", "if (r < -128.0) r = -128.0;"),
+    ("qb_127", "const double Qb = 128.0;\n    for (int64_t m = 0; m < M; ++m) {\n        const uint16_t",
+     "const double Qb = 127.0;\n    for (int64_t m = 0; m < M; ++m) {\n        const uint16_t"),
+    ("rescale_without_qb", "* beta * gamma[m] / Qb;", "* beta * gamma[m];"),
+    ("rescale_without_gamma", "* beta * gamma[m] / Qb;", "* beta / Qb;"),
+    ("acc_sign_ignored", "acc += (int64_t)packed_sign(packed, K, j, k) * (int64_t)xq[m * K + k];",
+     "acc += (int64_t)xq[m * K + k];"),
+    ("w1a1_and_not_xnor", "s += (int64_t)packed_sign(a, K, m, k) * (int64_t)packed_sign(b, K, j, k);",
+     "s += (packed_sign(a, K, m, k) == 1 && packed_sign(b, K, j, k) == 1) ? 1 : -1;"),
+    ("bf16_decode_wrong_half", "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+]
+
+
+@pytest.fixture(scope="module")
+def workdir():
+    d = tempfile.mkdtemp(prefix="oracle_mutants_")
+    yield d
+    shutil.rmtree(d, ignore_errors=True)
+
+
+def test_real_oracle_passes_every_pin(oracle):
+    assert pins.run_pins(oracle) == []
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(workdir, name, old, new):
+    text = open(SRC).read()
+    assert text.count(old) >= 1, f"pattern for {name} not found in oracle.c"
+    src = os.path.join(workdir, f"{name}.c")
+    with open(src, "w") as f:
+        f.write(text.replace(old, new))
+    lib = oracle_build.build(src, os.path.join(workdir, f"{name}.so"), strict=False)
+    failures = pins.run_pins(oracle_pkg.Oracle(lib))
+    assert failures, f"no pin caught the planted mistake {name}"
