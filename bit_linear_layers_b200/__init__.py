@@ -1,0 +1,195 @@
+"""Binarized linear layers on NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libbitlinear.so`` (C ABI in ``include/bitlinear.h``).
+Each function marshals torch tensors into device pointers and the current
+CUDA stream and calls the entry point of the same name; every step of the
+computation runs in the library's CUDA kernels. There is no CPU fallback:
+if the library is missing, importing the binding raises.
+
+    bin_pack(W, mode)                      -> packed, alpha[, beta]
+    bin_linear_w1a16(x, packed, alpha)     -> y (bf16)
+    bitlinear_w1a8(x, packed, beta)        -> y (fp32)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitlinear.so")
+
+BL_OK = 0
+BL_ERR_INVALID_ARG = -1
+BL_ERR_UNSUPPORTED = -2
+BL_ERR_CUDA = -3
+BL_ERR_TIMEOUT = -4
+BL_ERR_NO_DEVICE = -5
+
+BL_PACK_FBI = 0
+BL_PACK_BITNET = 1
+
+BL_OP_PACK_FBI = 0
+BL_OP_PACK_BITNET = 1
+BL_OP_W1A16 = 2
+BL_OP_W1A8 = 3
+
+# every symbol include/bitlinear.h declares, with its ctypes signature
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+_int = ctypes.c_int
+_sz = ctypes.c_size_t
+SIGNATURES = {
+    "bl_abi_version": ([], _int),
+    "bl_status_string": ([_int], ctypes.c_char_p),
+    "bl_workspace_bytes": ([_int, _i64, _i64, _i64], _sz),
+    "bin_pack": ([_p, _i64, _i64, _int, _p, _p, _p, _p, _sz, _p], _int),
+    "bin_linear_w1a16": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
+    "bitlinear_w1a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
+    "bitlinear_w1a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
+    "bl_device_error": ([_p, _int, ctypes.POINTER(_int)], _int),
+}
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, name: str, status: int):
+        self.status = status
+        super().__init__(f"{name} failed: {status} ({status_string(status)})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m bit_linear_layers_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.bl_status_string(int(status)).decode()
+
+
+def workspace_bytes(op: int, M: int, N: int, K: int) -> int:
+    return int(lib.bl_workspace_bytes(int(op), int(M), int(N), int(K)))
+
+
+def _check(name: str, rc: int) -> None:
+    if rc != BL_OK:
+        raise BitLinearError(name, rc)
+
+
+def _dev_ptr(t: torch.Tensor | None, dtype: torch.dtype, name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _workspace(op, M, N, K, device, ws):
+    need = workspace_bytes(op, M, N, K)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws, need
+
+
+# ---------------------------------------------------------------- entry points
+
+
+def bin_pack(W: torch.Tensor, mode: int = BL_PACK_FBI, *, packed=None, alpha=None, beta=None,
+             ws=None):
+    """Binarise W [N, K] fp32 into packed signs [N, K/32] int32 (bit patterns)
+    and scales. FBI: returns (packed, alpha[N]). BitNet: returns
+    (packed, alpha[1] = mean W, beta[1] = mean |W|)."""
+    N, K = W.shape
+    dev = W.device
+    if packed is None:
+        packed = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
+    if alpha is None:
+        alpha = torch.empty(N if mode == BL_PACK_FBI else 1, dtype=torch.float32, device=dev)
+    if mode == BL_PACK_BITNET and beta is None:
+        beta = torch.empty(1, dtype=torch.float32, device=dev)
+    op = BL_OP_PACK_BITNET if mode == BL_PACK_BITNET else BL_OP_PACK_FBI
+    ws, need = _workspace(op, 0, N, K, dev, ws)
+    rc = lib.bin_pack(_dev_ptr(W, torch.float32, "W"), N, K, int(mode),
+                      _dev_ptr(packed, torch.int32, "packed"), _dev_ptr(alpha, torch.float32, "alpha"),
+                      _dev_ptr(beta, torch.float32, "beta"), _dev_ptr(ws, torch.uint8, "ws"),
+                      ws.numel() if ws is not None else 0, _stream(dev))
+    _check("bin_pack", rc)
+    return (packed, alpha) if mode == BL_PACK_FBI else (packed, alpha, beta)
+
+
+def bin_linear_w1a16(x: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor, *, out=None):
+    """FBI-linear forward: y[m, j] = bf16(alpha[j] * sum_k sign_jk x[m, k])."""
+    M, K = x.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    rc = lib.bin_linear_w1a16(_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
+                              _dev_ptr(alpha, torch.float32, "alpha"),
+                              _dev_ptr(out, torch.bfloat16, "out"), M, N, K, _stream(x.device))
+    _check("bin_linear_w1a16", rc)
+    return out
+
+
+def bitlinear_w1a8(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, *, out=None, ws=None):
+    """BitNet BitLinear forward: LN, per-token absmax int8, +-1 GEMM, beta*gamma/128."""
+    M, K = x.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    ws, _ = _workspace(BL_OP_W1A8, M, N, K, x.device, ws)
+    rc = lib.bitlinear_w1a8(_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
+                            _dev_ptr(beta, torch.float32, "beta"), _dev_ptr(out, torch.float32, "out"),
+                            M, N, K, _dev_ptr(ws, torch.uint8, "ws"), ws.numel() if ws is not None else 0,
+                            _stream(x.device))
+    _check("bitlinear_w1a8", rc)
+    return out
+
+
+def bitlinear_w1a8_debug(x, packed, beta, *, xq_in=None, gamma_in=None, ws=None):
+    """As bitlinear_w1a8, also returning (xq int8 [M,K], gamma fp64 [M],
+    acc int32 [M,N]). With xq_in/gamma_in the LN/quant step is skipped."""
+    M, K = (xq_in.shape if xq_in is not None else x.shape)
+    N = packed.shape[0]
+    dev = packed.device
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    gamma = torch.empty(M, dtype=torch.float64, device=dev)
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev)
+    ws, _ = _workspace(BL_OP_W1A8, M, N, K, dev, ws)
+    rc = lib.bitlinear_w1a8_debug(
+        _dev_ptr(x, torch.bfloat16, "x") if x is not None else None,
+        _dev_ptr(packed, torch.int32, "packed"), _dev_ptr(beta, torch.float32, "beta"),
+        _dev_ptr(y, torch.float32, "y"), M, N, K, _dev_ptr(ws, torch.uint8, "ws"),
+        ws.numel() if ws is not None else 0, _dev_ptr(xq, torch.int8, "xq"),
+        _dev_ptr(gamma, torch.float64, "gamma"), _dev_ptr(acc, torch.int32, "acc"),
+        _dev_ptr(xq_in, torch.int8, "xq_in"), _dev_ptr(gamma_in, torch.float64, "gamma_in"),
+        _stream(dev))
+    _check("bitlinear_w1a8_debug", rc)
+    return y, xq, gamma, acc
+
+
+def device_error(clear: bool = True, device=None) -> tuple[int, int]:
+    """(status, where) of the first in-kernel fault on the current device."""
+    where = ctypes.c_int(0)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    rc = lib.bl_device_error(_stream(dev), int(bool(clear)), ctypes.byref(where))
+    return int(rc), int(where.value)

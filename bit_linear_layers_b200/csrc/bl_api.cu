@@ -1,0 +1,291 @@
+// libbitlinear.so: the C ABI declared in include/bitlinear.h.
+//
+// Host side only: argument validation, per-device one-time set-up, TMA
+// descriptor encoding and kernel dispatch. All kernels live in the headers
+// included below, so the library is one translation unit (no relocatable
+// device code). Nothing here allocates memory.
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "bitlinear.h"
+#include "bl_common.cuh"
+#include "bl_gemm.cuh"
+#include "bl_gemv.cuh"
+#include "bl_lnquant.cuh"
+#include "bl_pack.cuh"
+
+namespace bl {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxProduct = int64_t(1) << 40;
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---- per-device set-up ------------------------------------------------------
+struct DeviceState {
+  std::once_flag once;
+  int status = BL_ERR_NO_DEVICE;
+  int num_sms = 0;
+};
+DeviceState g_devices[kMaxDevices];
+
+template <typename Kernel>
+bool set_smem(Kernel k, int bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+int device_setup(int* num_sms) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return BL_ERR_NO_DEVICE;
+  }
+  DeviceState& st = g_devices[dev];
+  std::call_once(st.once, [&st, dev] {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10) {
+      cudaGetLastError();
+      st.status = BL_ERR_NO_DEVICE;
+      return;
+    }
+    st.num_sms = prop.multiProcessorCount;
+    bool ok = set_smem(gemm_bin_kernel<0>, GemmLayout<0>::SMEM_BYTES) &&
+              set_smem(gemm_bin_kernel<1>, GemmLayout<1>::SMEM_BYTES) &&
+              set_smem(gemv_w1a16_kernel<1>, gemv_smem_bytes(1)) &&
+              set_smem(gemv_w1a16_kernel<2>, gemv_smem_bytes(2)) &&
+              set_smem(gemv_w1a16_kernel<4>, gemv_smem_bytes(4));
+    if (!ok) cudaGetLastError();
+    st.status = ok ? BL_OK : BL_ERR_CUDA;
+  });
+  if (num_sms) *num_sms = st.num_sms;
+  return st.status;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+// ---- TMA descriptors ----------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `dtype`, box [box_rows][box_cols].
+bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                 uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                 CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int check_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 1 || K < 1) return BL_ERR_INVALID_ARG;
+  if (K % 128 != 0) return BL_ERR_UNSUPPORTED;
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return BL_ERR_UNSUPPORTED;
+  if (M * K >= kMaxProduct || N * K >= kMaxProduct || M * N >= kMaxProduct) return BL_ERR_UNSUPPORTED;
+  return BL_OK;
+}
+
+// ---- W1A8 shared body -----------------------------------------------------------
+int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
+              int64_t N, int64_t K, void* ws, size_t ws_bytes, int8_t* xq_out, double* gamma_out,
+              int32_t* acc_out, const int8_t* xq_in, const double* gamma_in, void* stream) {
+  int rc = check_shape(M, N, K);
+  if (rc != BL_OK) return rc;
+  if (M == 0) return BL_OK;
+  if (!packed || !beta || !y || !aligned16(packed) || !aligned16(y)) return BL_ERR_INVALID_ARG;
+  if (xq_in) {
+    if (!gamma_in || !aligned16(xq_in)) return BL_ERR_INVALID_ARG;
+  } else {
+    if (!x || !aligned16(x)) return BL_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws) || ws_bytes < bl_workspace_bytes(BL_OP_W1A8, M, N, K))
+      return BL_ERR_INVALID_ARG;
+  }
+  rc = device_setup(nullptr);
+  if (rc != BL_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const int8_t* codes = xq_in;
+  const double* gam = gamma_in;
+  if (!xq_in) {
+    int8_t* xq_ws = static_cast<int8_t*>(ws);
+    double* g_ws = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(size_t(M * K)));
+    ln_quant_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, K, xq_ws, g_ws);
+    if ((rc = launch_status()) != BL_OK) return rc;
+    codes = xq_ws;
+    gam = g_ws;
+  }
+  if (xq_out && cudaMemcpyAsync(xq_out, codes, size_t(M * K), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return BL_ERR_CUDA;
+  if (gamma_out &&
+      cudaMemcpyAsync(gamma_out, gam, size_t(M) * sizeof(double), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return BL_ERR_CUDA;
+
+  if (M <= 16) {
+    const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
+    if (M <= 4)
+      gemv_w1a8_kernel<4><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+    else if (M <= 8)
+      gemv_w1a8_kernel<8><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+    else
+      gemv_w1a8_kernel<16><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+    return launch_status();
+  }
+  CUtensorMap tm_a, tm_bits;
+  if (!make_map_2d(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(K), uint64_t(M), 128, kBM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4,
+                   GemmCfg<1>::BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BL_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(cdiv(N, GemmCfg<1>::BN)), static_cast<unsigned>(cdiv(M, kBM)));
+  gemm_bin_kernel<1><<<grid, kGemmThreads, GemmLayout<1>::SMEM_BYTES, s>>>(
+      tm_a, tm_bits, int(M), int(N), int(K), nullptr, gam, beta, y, acc_out);
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace bl
+
+using namespace bl;
+
+extern "C" {
+
+int bl_abi_version(void) { return 1; }
+
+const char* bl_status_string(int status) {
+  switch (status) {
+    case BL_OK: return "ok";
+    case BL_ERR_INVALID_ARG: return "invalid argument (null, negative size, misaligned or short workspace)";
+    case BL_ERR_UNSUPPORTED: return "unsupported shape (K must be a positive multiple of 128; sizes below 2^31, products below 2^40)";
+    case BL_ERR_CUDA: return "CUDA runtime or launch error";
+    case BL_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+    case BL_ERR_NO_DEVICE: return "no usable sm_100 device is current";
+    default: return "unknown status";
+  }
+}
+
+size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  switch (op) {
+    case BL_OP_PACK_BITNET: return align256(size_t(N) * 2 * sizeof(double)) + 256;
+    case BL_OP_W1A8: return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double));
+    default: return 0;
+  }
+}
+
+int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, float* alpha,
+             float* beta, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_shape(0, N, K);
+  if (rc != BL_OK) return rc;
+  if (mode != BL_PACK_FBI && mode != BL_PACK_BITNET) return BL_ERR_INVALID_ARG;
+  if (!W || !packed || !alpha || !aligned16(W) || !aligned16(packed)) return BL_ERR_INVALID_ARG;
+  if (mode == BL_PACK_BITNET &&
+      (!beta || !ws || !aligned16(ws) || ws_bytes < bl_workspace_bytes(BL_OP_PACK_BITNET, 0, N, K)))
+    return BL_ERR_INVALID_ARG;
+  int sms = 0;
+  rc = device_setup(&sms);
+  if (rc != BL_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t warps_per_block = kPackThreads / 32;
+  const unsigned grid = static_cast<unsigned>(
+      cdiv(N, warps_per_block) < int64_t(sms) * 16 ? cdiv(N, warps_per_block) : int64_t(sms) * 16);
+  if (mode == BL_PACK_FBI) {
+    pack_rows_kernel<false><<<grid, kPackThreads, 0, s>>>(W, N, K, packed, alpha, nullptr);
+    return launch_status();
+  }
+  double* sums = static_cast<double*>(ws);
+  double* scalars = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(size_t(N) * 2 * sizeof(double)));
+  row_sums_kernel<<<grid, kPackThreads, 0, s>>>(W, N, K, sums);
+  if ((rc = launch_status()) != BL_OK) return rc;
+  global_scalars_kernel<<<1, kReduceThreads, 0, s>>>(sums, N, K, scalars, alpha, beta);
+  if ((rc = launch_status()) != BL_OK) return rc;
+  pack_rows_kernel<true><<<grid, kPackThreads, 0, s>>>(W, N, K, packed, nullptr, scalars);
+  return launch_status();
+}
+
+int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
+                     int64_t M, int64_t N, int64_t K, void* stream) {
+  int rc = check_shape(M, N, K);
+  if (rc != BL_OK) return rc;
+  if (M == 0) return BL_OK;
+  if (!x || !packed || !alpha || !y || !aligned16(x) || !aligned16(packed) || !aligned16(y))
+    return BL_ERR_INVALID_ARG;
+  rc = device_setup(nullptr);
+  if (rc != BL_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M <= 4) {
+    const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
+    if (M == 1)
+      gemv_w1a16_kernel<1><<<grid, kGemvThreads, gemv_smem_bytes(1), s>>>(x, packed, alpha, y, int(M), N, K);
+    else if (M == 2)
+      gemv_w1a16_kernel<2><<<grid, kGemvThreads, gemv_smem_bytes(2), s>>>(x, packed, alpha, y, int(M), N, K);
+    else
+      gemv_w1a16_kernel<4><<<grid, kGemvThreads, gemv_smem_bytes(4), s>>>(x, packed, alpha, y, int(M), N, K);
+    return launch_status();
+  }
+  CUtensorMap tm_a, tm_bits;
+  if (!make_map_2d(&tm_a, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(K), uint64_t(M), 64, kBM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4,
+                   GemmCfg<0>::BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BL_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(cdiv(N, GemmCfg<0>::BN)), static_cast<unsigned>(cdiv(M, kBM)));
+  gemm_bin_kernel<0><<<grid, kGemmThreads, GemmLayout<0>::SMEM_BYTES, s>>>(
+      tm_a, tm_bits, int(M), int(N), int(K), alpha, nullptr, nullptr, y, nullptr);
+  return launch_status();
+}
+
+int bitlinear_w1a8(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
+                   int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream) {
+  return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, nullptr, nullptr, nullptr, nullptr,
+                   nullptr, stream);
+}
+
+int bitlinear_w1a8_debug(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                         int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes, int8_t* xq_out,
+                         double* gamma_out, int32_t* acc_out, const int8_t* xq_in,
+                         const double* gamma_in, void* stream) {
+  return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, xq_out, gamma_out, acc_out, xq_in,
+                   gamma_in, stream);
+}
+
+int bl_device_error(void* stream, int clear, int* where_out) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BL_ERR_CUDA;
+  DeviceError e{0, 0};
+  if (cudaMemcpyFromSymbol(&e, g_device_error, sizeof e) != cudaSuccess) return BL_ERR_CUDA;
+  if (clear) {
+    const DeviceError z{0, 0};
+    if (cudaMemcpyToSymbol(g_device_error, &z, sizeof z) != cudaSuccess) return BL_ERR_CUDA;
+  }
+  if (where_out) *where_out = e.where;
+  return e.code;
+}
+
+}  // extern "C"

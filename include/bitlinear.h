@@ -1,0 +1,149 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so: binarized linear layers on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Two layers and the step that feeds them:
+ *   - FBI-linear (W1A16): "FBI-LLM: Fully Binarized Large Language Model"
+ *     (MarkTechPost article as rewritten on cloudsagepro.com), the paragraph
+ *     defining FBI-linear and the experiments paragraph (W1A16).
+ *   - BitLinear (W1A8): "BitNet b1.58: 1bit LLM 时代" (coreui.cn), section 1
+ *     (BitNet), Eq.(1)-(8).
+ *   - bin_pack: the binarisation of those two passages (sign of W, or of
+ *     W minus its mean) written as 1-bit planes plus the scales.
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent)
+ *     unless a parameter says otherwise. The caller owns every buffer; the
+ *     library allocates nothing on any call path.
+ *   - Layouts are row-major and dense. Activations x are bf16, passed as raw
+ *     16-bit patterns (uint16_t). Weights W are fp32.
+ *   - Packed sign planes: row j of an N x K sign matrix is K/32 uint32 words;
+ *     element (j,k) is bit (k mod 32) of word [j*(K/32) + k/32]; a set bit is
+ *     +1, a clear bit -1. (The pages give no layout; this is the library's.)
+ *   - Shapes: M >= 0 tokens, N >= 1 output channels, K >= 128 inputs with
+ *     K % 128 == 0 (so a packed row is a whole number of 16-byte chunks).
+ *     M == 0 is a valid no-op. Every pointer must be 16-byte aligned.
+ *     M*K, N*K and M*N must each be below 2^40.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and never synchronise it. Argument errors are returned
+ *     before anything is enqueued. Launch errors are returned as
+ *     BL_ERR_CUDA. Faults detected inside a kernel (a bounded wait that ran
+ *     out) are recorded in a per-device error word, read by bl_device_error.
+ *   - No C++ exception crosses this boundary. Thread-safe: the library keeps
+ *     no mutable host state apart from per-device one-time set-up.
+ *   - Buffers passed to one call must not overlap, except that inputs may
+ *     alias other inputs.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define BL_OK 0
+#define BL_ERR_INVALID_ARG (-1) /* null pointer, negative size, misalignment    */
+#define BL_ERR_UNSUPPORTED (-2) /* shape outside the supported set (K % 128)     */
+#define BL_ERR_CUDA (-3)        /* a CUDA runtime/driver call or launch failed   */
+#define BL_ERR_TIMEOUT (-4)     /* a kernel's bounded wait ran out (device word) */
+#define BL_ERR_NO_DEVICE (-5)   /* no usable sm_100 device is current            */
+
+/* ---- bin_pack modes ----------------------------------------------------- */
+#define BL_PACK_FBI 0    /* sign(W), per-output-channel alpha                 */
+#define BL_PACK_BITNET 1 /* sign(W - mean W), global alpha and beta           */
+
+/* ---- ops for bl_workspace_bytes ----------------------------------------- */
+#define BL_OP_PACK_FBI 0
+#define BL_OP_PACK_BITNET 1
+#define BL_OP_W1A16 2
+#define BL_OP_W1A8 3
+
+/* Library ABI version (this header: 1). */
+int bl_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* bl_status_string(int status);
+
+/* Bytes of device workspace the call `op` needs for the given shape (0 when
+ * it needs none). Host-only: touches no device. Returns 0 for invalid
+ * shapes too; the call itself reports those. */
+size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
+
+/*
+ * bin_pack -- binarise W [N x K] fp32 into packed sign planes plus scales.
+ *
+ * mode BL_PACK_FBI ("FBI-LLM" page, FBI-linear paragraph):
+ *   s_jk = Sign(W_jk) with Sign(v) = +1 if v > 0 else -1 (BitNet Eq.(2));
+ *   alpha[j] = (1/K) * sum_k |W_jk|  -- one scale per output channel,
+ *   accumulated in fp64 and rounded once to fp32. `alpha` has N floats.
+ *   `beta` is unused (may be NULL). No workspace (ws may be NULL).
+ * mode BL_PACK_BITNET ("BitNet b1.58" page, section 1, Eq.(1)-(3), (8)):
+ *   a = (1/NK) * sum W (fp64);  s_jk = Sign(W_jk - a) compared in fp64;
+ *   beta = (1/NK) * sum |W| (fp64, unshifted W).
+ *   alpha[0] = (float)a (informational), beta[0] = (float)beta.
+ *   Needs ws of bl_workspace_bytes(BL_OP_PACK_BITNET, 0, N, K) bytes.
+ * Outputs: packed [N x K/32] uint32 (layout above). All device pointers.
+ */
+int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, float* alpha,
+             float* beta, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bin_linear_w1a16 -- FBI-linear forward, 1-bit weights, bf16 activations
+ * ("FBI-LLM" page: sign(W) times a full-precision per-output-channel scale;
+ * W1A16 configuration of its experiments paragraph):
+ *   y[m][j] = bf16( alpha[j] * sum_k s_jk * x[m][k] )
+ * x [M x K] bf16, packed [N x K/32], alpha [N] fp32 (any values: the page
+ * only initialises them), y [M x N] bf16 (round to nearest even).
+ * Accumulation is fp32. Decode-sized M uses a bandwidth-bound GEMV kernel,
+ * larger M a tcgen05 tensor-core GEMM. No workspace.
+ */
+int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
+                     int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * bitlinear_w1a8 -- BitNet BitLinear forward ("BitNet b1.58" page,
+ * section 1, Eq.(4)-(5), (7)-(8)), per token m:
+ *   mu = mean_k x,  var = mean_k (x - mu)^2,  ln_k = (x_k - mu)/sqrt(var + 1e-5)
+ *   gamma_m = max_k |ln_k|
+ *   q_mk = clamp(round_half_even(ln_k * 128 / gamma_m), -127, 127)  (0 if gamma_m == 0)
+ *   acc[m][j] = sum_k s_jk * q_mk        (exact int32)
+ *   y[m][j] = fp32( acc * beta * gamma_m / 128 )   (evaluated in fp64)
+ * LN statistics and the quantisation decision are taken in fp64.
+ * x [M x K] bf16, packed [N x K/32] (from BL_PACK_BITNET), beta: DEVICE
+ * pointer to one float (so pack -> forward needs no host round trip),
+ * y [M x N] fp32. Needs ws of bl_workspace_bytes(BL_OP_W1A8, M, N, K) bytes
+ * (the int8 codes and per-token gamma live there between the two kernels).
+ */
+int bitlinear_w1a8(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                   int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bitlinear_w1a8_debug -- the same kernels as bitlinear_w1a8, also exporting
+ * the intermediates for two-level parity checks. Any of the extra outputs
+ * may be NULL. xq_out [M x K] int8 codes, gamma_out [M] fp64, acc_out
+ * [M x N] int32 accumulators. If xq_in is non-NULL the LN/quantisation step
+ * is skipped and (xq_in [M x K] int8, gamma_in [M] fp64) are used instead.
+ */
+int bitlinear_w1a8_debug(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                         int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
+                         int8_t* xq_out, double* gamma_out, int32_t* acc_out,
+                         const int8_t* xq_in, const double* gamma_in, void* stream);
+
+/*
+ * bl_device_error -- synchronise `stream`, then return the first in-kernel
+ * fault recorded on the current device since the last clear (BL_OK if none;
+ * BL_ERR_TIMEOUT when a bounded wait ran out). If `clear` is non-zero the
+ * word is reset. `where_out` (host pointer, may be NULL) receives a code
+ * naming the kernel and wait that gave up.
+ */
+int bl_device_error(void* stream, int clear, int* where_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

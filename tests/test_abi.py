@@ -1,0 +1,96 @@
+"""The C ABI library without a GPU: it loads, exports every function the
+header declares, and rejects bad arguments on the host before touching a
+device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("bin_pack", "bin_linear_w1a16", "bitlinear_w1a8", "bitlinear_w1a8_debug",
+              "bl_workspace_bytes", "bl_status_string", "bl_device_error", "bl_abi_version"):
+        assert n in names, names
+
+
+def test_library_exports_every_declared_symbol():
+    import bit_linear_layers_b200 as bl
+    raw = ctypes.CDLL(bl.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), f"{name} declared in bitlinear.h but not exported"
+    assert set(declared_functions()) == set(bl.SIGNATURES), "binding and header disagree"
+
+
+def test_abi_version_and_status_strings():
+    import bit_linear_layers_b200 as bl
+    assert bl.lib.bl_abi_version() == 1
+    for code in (0, -1, -2, -3, -4, -5):
+        s = bl.status_string(code)
+        assert s and s != "unknown status"
+    assert bl.status_string(12345) == "unknown status"
+
+
+def test_workspace_sizes():
+    import bit_linear_layers_b200 as bl
+    assert bl.workspace_bytes(bl.BL_OP_PACK_FBI, 0, 4096, 4096) == 0
+    assert bl.workspace_bytes(bl.BL_OP_W1A16, 16, 4096, 4096) == 0
+    assert bl.workspace_bytes(bl.BL_OP_PACK_BITNET, 0, 4096, 4096) >= 4096 * 16 + 16
+    ws = bl.workspace_bytes(bl.BL_OP_W1A8, 512, 5632, 2048)
+    assert ws >= 512 * 2048 + 512 * 8 and ws % 256 == 0
+    assert bl.workspace_bytes(bl.BL_OP_W1A8, -1, 1, 128) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case below fails validation
+ODD = ctypes.c_void_p(0x10001)
+
+
+@pytest.mark.parametrize("M,N,K,code", [
+    (1, 64, 100, -2),      # K not a multiple of 128
+    (1, 64, 0, -1),        # K < 1
+    (-1, 64, 128, -1),     # negative M
+    (1, 0, 128, -1),       # N < 1
+    (1 << 31, 1, 128, -2),  # M beyond int32
+])
+def test_w1a16_shape_validation(M, N, K, code):
+    import bit_linear_layers_b200 as bl
+    assert bl.lib.bin_linear_w1a16(FAKE, FAKE, FAKE, FAKE, M, N, K, None) == code
+
+
+def test_null_and_misaligned_pointers_rejected():
+    import bit_linear_layers_b200 as bl
+    assert bl.lib.bin_linear_w1a16(None, FAKE, FAKE, FAKE, 1, 128, 128, None) == -1
+    assert bl.lib.bin_linear_w1a16(ODD, FAKE, FAKE, FAKE, 1, 128, 128, None) == -1
+    assert bl.lib.bitlinear_w1a8(FAKE, FAKE, None, FAKE, 1, 128, 128, FAKE, 1 << 20, None) == -1
+    # workspace too small
+    assert bl.lib.bitlinear_w1a8(FAKE, FAKE, FAKE, FAKE, 4, 128, 128, FAKE, 16, None) == -1
+    assert bl.lib.bin_pack(FAKE, 128, 128, 7, FAKE, FAKE, FAKE, None, 0, None) == -1
+    assert bl.lib.bin_pack(FAKE, 128, 128, bl.BL_PACK_BITNET, FAKE, FAKE, FAKE, None, 0, None) == -1
+    assert bl.lib.bin_pack(FAKE, 128, 96, bl.BL_PACK_FBI, FAKE, FAKE, None, None, 0, None) == -2
+
+
+def test_zero_tokens_is_a_noop():
+    import bit_linear_layers_b200 as bl
+    assert bl.lib.bin_linear_w1a16(None, FAKE, FAKE, None, 0, 128, 128, None) == 0
+    assert bl.lib.bitlinear_w1a8(None, FAKE, FAKE, FAKE, 0, 128, 128, None, 0, None) == 0
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The CUDA binding and sources never reference the oracle."""
+    pkg = os.path.join(ROOT, "bit_linear_layers_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "liboracle" not in text and "oracle.c" not in text, f
