@@ -61,7 +61,7 @@ class BitLinearError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m bit_linear_layers_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python bit_linear_layers_b200/build.py` "
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (args, res) in SIGNATURES.items():

@@ -1,6 +1,8 @@
 """Build ``libbitlinear.so`` in-tree for sm_100a with nvcc.
 
-    python -m bit_linear_layers_b200.build [--verbose-ptxas]
+    python bit_linear_layers_b200/build.py [--verbose-ptxas]
+
+(Run it by path: importing the package loads the library it builds.)
 
 nvcc cross-compiles, so this runs on machines without a GPU.
 """
