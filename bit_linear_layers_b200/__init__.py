@@ -26,6 +26,8 @@ BL_ERR_UNSUPPORTED = -2
 BL_ERR_CUDA = -3
 BL_ERR_TIMEOUT = -4
 BL_ERR_NO_DEVICE = -5
+BL_ERR_SCRATCH_LIMIT = -6
+W1A8_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 BL_PACK_FBI = 0
 BL_PACK_BITNET = 1
@@ -49,6 +51,7 @@ SIGNATURES = {
     "bitlinear_w1a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w1a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
     "bl_device_error": ([_p, _int, ctypes.POINTER(_int)], _int),
+    "bitlinear_w1a8_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
 }
 
 
@@ -185,6 +188,22 @@ def bitlinear_w1a8_debug(x, packed, beta, *, xq_in=None, gamma_in=None, ws=None)
         _stream(dev))
     _check("bitlinear_w1a8_debug", rc)
     return y, xq, gamma, acc
+
+
+def bitlinear_w1a8_noalloc(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, *, out=None):
+    """bitlinear_w1a8 without a workspace, for callers that cannot allocate
+    device memory while they run: the codes and gamma live in a fixed 4 MiB
+    scratch array inside the library (bl_workspace_bytes(BL_OP_W1A8, M, N, K)
+    must fit in it). Calls that overlap on the GPU share that array and race."""
+    M, K = x.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    rc = lib.bitlinear_w1a8_noalloc(_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
+                                    _dev_ptr(beta, torch.float32, "beta"), _dev_ptr(out, torch.float32, "out"),
+                                    M, N, K, _stream(x.device))
+    _check("bitlinear_w1a8_noalloc", rc)
+    return out
 
 
 def device_error(clear: bool = True, device=None) -> tuple[int, int]:

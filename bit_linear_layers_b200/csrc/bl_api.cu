@@ -187,6 +187,9 @@ const char* bl_status_string(int status) {
     case BL_ERR_CUDA: return "CUDA runtime or launch error";
     case BL_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
     case BL_ERR_NO_DEVICE: return "no usable sm_100 device is current";
+    case BL_ERR_SCRATCH_LIMIT:
+      return "problem exceeds the fixed scratch of bitlinear_w1a8_noalloc "
+             "(bl_workspace_bytes(BL_OP_W1A8, M, N, K) must be at most 4 MiB)";
     default: return "unknown status";
   }
 }
@@ -289,3 +292,64 @@ int bl_device_error(void* stream, int clear, int* where_out) {
 }
 
 }  // extern "C"
+
+// ---- allocation-free BitLinear ------------------------------------------------
+// bitlinear_w1a8_noalloc serves callers that cannot allocate device memory:
+// operators embedded in a host framework that only hands them their inputs
+// and outputs, and loops with a fixed up-front memory plan that must not call
+// cudaMalloc while running. It runs the same LN/quant and GEMM kernels as
+// bitlinear_w1a8, with the codes and gamma kept in the array below instead
+// of a caller workspace.
+namespace bl {
+namespace {
+
+// Lives on every device that loads this library, until the process exits.
+static __device__ __align__(256) uint8_t g_w1a8_noalloc_scratch[BL_W1A8_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocScratch {
+  std::once_flag once;
+  void* ptr = nullptr;
+  int status = BL_ERR_NO_DEVICE;
+};
+NoallocScratch g_noalloc[kMaxDevices];
+
+// Device address of the scratch array on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return BL_ERR_NO_DEVICE;
+  }
+  NoallocScratch& st = g_noalloc[dev];
+  std::call_once(st.once, [&st] {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_w1a8_noalloc_scratch) == cudaSuccess && p != nullptr) {
+      st.ptr = p;
+      st.status = BL_OK;
+    } else {
+      cudaGetLastError();
+      st.status = BL_ERR_CUDA;
+    }
+  });
+  *out = st.ptr;
+  return st.status;
+}
+
+}  // namespace
+}  // namespace bl
+
+extern "C" int bitlinear_w1a8_noalloc(const uint16_t* x, const uint32_t* packed, const float* beta,
+                                      float* y, int64_t M, int64_t N, int64_t K, void* stream) {
+  int rc = check_shape(M, N, K);
+  if (rc != BL_OK) return rc;
+  if (M == 0) return BL_OK;
+  if (bl_workspace_bytes(BL_OP_W1A8, M, N, K) > BL_W1A8_NOALLOC_SCRATCH_BYTES) return BL_ERR_SCRATCH_LIMIT;
+  if (!x || !packed || !beta || !y) return BL_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != BL_OK) return rc;
+  return w1a8_impl(x, packed, beta, y, M, N, K, scratch, BL_W1A8_NOALLOC_SCRATCH_BYTES, nullptr,
+                   nullptr, nullptr, nullptr, nullptr, stream);
+}

@@ -51,6 +51,8 @@ extern "C" {
 #define BL_ERR_CUDA (-3)        /* a CUDA runtime/driver call or launch failed   */
 #define BL_ERR_TIMEOUT (-4)     /* a kernel's bounded wait ran out (device word) */
 #define BL_ERR_NO_DEVICE (-5)   /* no usable sm_100 device is current            */
+#define BL_ERR_SCRATCH_LIMIT (-6) /* problem too big for the fixed scratch of       */
+                                  /* bitlinear_w1a8_noalloc                         */
 
 /* ---- bin_pack modes ----------------------------------------------------- */
 #define BL_PACK_FBI 0    /* sign(W), per-output-channel alpha                 */
@@ -141,6 +143,36 @@ int bitlinear_w1a8_debug(const uint16_t* x, const uint32_t* packed, const float*
  * naming the kernel and wait that gave up.
  */
 int bl_device_error(void* stream, int clear, int* where_out);
+
+/*
+ * bitlinear_w1a8_noalloc -- bitlinear_w1a8 for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this call: it exists for users of the
+ * library, not for the method. Some callers cannot hand the layer a
+ * workspace: an operator plugged into a host framework that passes it only
+ * its input and output buffers, or an inference loop whose device memory is
+ * planned once up front and which may not call cudaMalloc while it runs
+ * (cudaMalloc can synchronise the device and stall other work). This entry
+ * point runs the same kernels as bitlinear_w1a8 but keeps the int8 codes and
+ * per-token gamma in a fixed scratch array that lives inside the library
+ * (BL_W1A8_NOALLOC_SCRATCH_BYTES per device, held by every GPU that loads
+ * the library until the process exits). It calls no allocator.
+ *
+ * Limit: bl_workspace_bytes(BL_OP_W1A8, M, N, K) must not exceed
+ * BL_W1A8_NOALLOC_SCRATCH_BYTES (about M*K + 8*M bytes; e.g. 512 tokens of
+ * K = 5632 fit), else BL_ERR_SCRATCH_LIMIT is returned and nothing runs.
+ * Arguments and results are otherwise those of bitlinear_w1a8.
+ *
+ * The first call on a device looks up the scratch array's device address
+ * (once per device, with that device current); make that first call before
+ * any stream capture. All calls on a device share the one array and it keeps
+ * the last call's contents; nothing in it needs to start at zero (each call
+ * overwrites every byte it later reads), but calls whose kernels overlap on
+ * the GPU (different streams, no ordering between them) race on it.
+ */
+#define BL_W1A8_NOALLOC_SCRATCH_BYTES (4u << 20)
+int bitlinear_w1a8_noalloc(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                           int64_t M, int64_t N, int64_t K, void* stream);
 
 #ifdef __cplusplus
 }
