@@ -29,6 +29,8 @@ BL_ERR_NO_DEVICE = -5
 BL_ERR_SCRATCH_LIMIT = -6
 W1A8_NOALLOC_SCRATCH_BYTES = 4 << 20
 
+BL_FLAG_OVERLAP_PREVIOUS = 1
+
 BL_PACK_FBI = 0
 BL_PACK_BITNET = 1
 
@@ -48,6 +50,7 @@ SIGNATURES = {
     "bl_workspace_bytes": ([_int, _i64, _i64, _i64], _sz),
     "bin_pack": ([_p, _i64, _i64, _int, _p, _p, _p, _p, _sz, _p], _int),
     "bin_linear_w1a16": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
+    "bin_linear_w1a16_ex": ([_p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_uint, _p], _int),
     "bitlinear_w1a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w1a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
     "bl_device_error": ([_p, _int, ctypes.POINTER(_int)], _int),
@@ -139,16 +142,24 @@ def bin_pack(W: torch.Tensor, mode: int = BL_PACK_FBI, *, packed=None, alpha=Non
     return (packed, alpha) if mode == BL_PACK_FBI else (packed, alpha, beta)
 
 
-def bin_linear_w1a16(x: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor, *, out=None):
-    """FBI-linear forward: y[m, j] = bf16(alpha[j] * sum_k sign_jk x[m, k])."""
+def bin_linear_w1a16(x: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor, *, out=None,
+                     flags: int = 0):
+    """FBI-linear forward: y[m, j] = bf16(alpha[j] * sum_k sign_jk x[m, k]).
+    ``flags`` (bin_linear_w1a16_ex): BL_FLAG_OVERLAP_PREVIOUS lets the
+    single-token kernel stream its weights while the previous kernel on the
+    stream finishes; only valid when that kernel does not write them."""
     M, K = x.shape
     N = packed.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    rc = lib.bin_linear_w1a16(_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
-                              _dev_ptr(alpha, torch.float32, "alpha"),
-                              _dev_ptr(out, torch.bfloat16, "out"), M, N, K, _stream(x.device))
-    _check("bin_linear_w1a16", rc)
+    args = (_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
+            _dev_ptr(alpha, torch.float32, "alpha"), _dev_ptr(out, torch.bfloat16, "out"), M, N, K)
+    if flags:
+        rc = lib.bin_linear_w1a16_ex(*args, int(flags), _stream(x.device))
+        _check("bin_linear_w1a16_ex", rc)
+    else:
+        rc = lib.bin_linear_w1a16(*args, _stream(x.device))
+        _check("bin_linear_w1a16", rc)
     return out
 
 

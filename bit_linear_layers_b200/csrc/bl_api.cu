@@ -12,8 +12,9 @@
 
 #include "bitlinear.h"
 #include "bl_common.cuh"
-#include "bl_gemm.cuh"
+#include "bl_gemm_ts.cuh"
 #include "bl_gemv.cuh"
+#include "bl_gemv_lut.cuh"
 #include "bl_lnquant.cuh"
 #include "bl_pack.cuh"
 
@@ -56,11 +57,16 @@ int device_setup(int* num_sms) {
       return;
     }
     st.num_sms = prop.multiProcessorCount;
-    bool ok = set_smem(gemm_bin_kernel<0>, GemmLayout<0>::SMEM_BYTES) &&
-              set_smem(gemm_bin_kernel<1>, GemmLayout<1>::SMEM_BYTES) &&
-              set_smem(gemv_w1a16_kernel<1>, gemv_smem_bytes(1)) &&
+    bool ok = set_smem(gemv_w1a16_kernel<1>, gemv_smem_bytes(1)) &&
               set_smem(gemv_w1a16_kernel<2>, gemv_smem_bytes(2)) &&
-              set_smem(gemv_w1a16_kernel<4>, gemv_smem_bytes(4));
+              set_smem(gemv_w1a16_kernel<4>, gemv_smem_bytes(4)) &&
+              set_smem(gemv_w1a16_lut_kernel<1>, 1 * kLutPageBytes) &&
+              set_smem(gemv_w1a16_lut_kernel<2>, 2 * kLutPageBytes) &&
+              set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
+              set_smem(gemm_ts_kernel<0, 32>, TsCfg<0, 32>::SMEM_BYTES) &&
+              set_smem(gemm_ts_kernel<0, 128>, TsCfg<0, 128>::SMEM_BYTES) &&
+              set_smem(gemm_ts_kernel<1, 32>, TsCfg<1, 32>::SMEM_BYTES) &&
+              set_smem(gemm_ts_kernel<1, 128>, TsCfg<1, 128>::SMEM_BYTES);
     if (!ok) cudaGetLastError();
     st.status = ok ? BL_OK : BL_ERR_CUDA;
   });
@@ -113,6 +119,55 @@ int check_shape(int64_t M, int64_t N, int64_t K) {
   return BL_OK;
 }
 
+// ---- single-token lookup-table GEMV ------------------------------------------------
+template <int NP>
+cudaError_t launch_lut(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
+                       int N, int K, int C, int slice_words, bool overlap, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(C), static_cast<unsigned>(cdiv(N, kLutRowsPerCluster)), 1);
+  cfg.blockDim = dim3(kLutThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(NP) * kLutPageBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = static_cast<unsigned>(C);
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = overlap ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, gemv_w1a16_lut_kernel<NP>, x, packed, alpha, y, N, K, slice_words);
+}
+
+// ---- tensor-core GEMM with the signs in tensor memory ------------------------------
+// activations [M][K] (bf16 for KIND 0, int8 codes for KIND 1) x packed signs [N][K/32]
+template <int KIND, int T>
+int launch_ts(const void* act, const uint32_t* packed, int64_t M, int64_t N, int64_t K,
+              const float* alpha, const double* gamma, const float* beta, void* y, int32_t* acc_out,
+              int num_sms, cudaStream_t s) {
+  using C = TsCfg<KIND, T>;
+  CUtensorMap tm_x, tm_bits;
+  const bool ok =
+      make_map_2d(&tm_x, act, KIND == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                  C::ELEM, uint64_t(K), uint64_t(M), 128 / C::ELEM, T, CU_TENSOR_MAP_SWIZZLE_128B) &&
+      make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4,
+                  kTsRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return BL_ERR_CUDA;
+  // output tile written by one bulk tensor store when the row pitch allows it
+  CUtensorMap tm_y;
+  std::memset(&tm_y, 0, sizeof tm_y);
+  const int use_tma_store =
+      (N * C::OUT_ELEM) % 16 == 0 &&
+      make_map_2d(&tm_y, y, KIND == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  C::OUT_ELEM, uint64_t(N), uint64_t(M), kTsRows, T, CU_TENSOR_MAP_SWIZZLE_NONE);
+  const int64_t tiles = cdiv(M, T) * cdiv(N, kTsRows);
+  const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
+  gemm_ts_kernel<KIND, T><<<grid, kTsThreads, C::SMEM_BYTES, s>>>(
+      tm_x, tm_bits, tm_y, use_tma_store, int(M), int(N), int(K), alpha, gamma, beta, y, acc_out);
+  return launch_status();
+}
+
 // ---- W1A8 shared body -----------------------------------------------------------
 int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
               int64_t N, int64_t K, void* ws, size_t ws_bytes, int8_t* xq_out, double* gamma_out,
@@ -158,16 +213,11 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
       gemv_w1a8_kernel<16><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
     return launch_status();
   }
-  CUtensorMap tm_a, tm_bits;
-  if (!make_map_2d(&tm_a, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(K), uint64_t(M), 128, kBM,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4,
-                   GemmCfg<1>::BN, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return BL_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(cdiv(N, GemmCfg<1>::BN)), static_cast<unsigned>(cdiv(M, kBM)));
-  gemm_bin_kernel<1><<<grid, kGemmThreads, GemmLayout<1>::SMEM_BYTES, s>>>(
-      tm_a, tm_bits, int(M), int(N), int(K), nullptr, gam, beta, y, acc_out);
-  return launch_status();
+  int sms = 0;
+  device_setup(&sms);
+  if (M <= 32)
+    return launch_ts<1, 32>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s);
+  return launch_ts<1, 128>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s);
 }
 
 }  // namespace
@@ -235,33 +285,49 @@ int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, f
 
 int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
                      int64_t M, int64_t N, int64_t K, void* stream) {
+  return bin_linear_w1a16_ex(x, packed, alpha, y, M, N, K, 0u, stream);
+}
+
+int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
+                        int64_t M, int64_t N, int64_t K, unsigned flags, void* stream) {
   int rc = check_shape(M, N, K);
   if (rc != BL_OK) return rc;
+  if (flags & ~BL_FLAG_OVERLAP_PREVIOUS) return BL_ERR_INVALID_ARG;
   if (M == 0) return BL_OK;
   if (!x || !packed || !alpha || !y || !aligned16(x) || !aligned16(packed) || !aligned16(y))
     return BL_ERR_INVALID_ARG;
   rc = device_setup(nullptr);
   if (rc != BL_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M <= 4) {
-    const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
-    if (M == 1)
-      gemv_w1a16_kernel<1><<<grid, kGemvThreads, gemv_smem_bytes(1), s>>>(x, packed, alpha, y, int(M), N, K);
-    else if (M == 2)
-      gemv_w1a16_kernel<2><<<grid, kGemvThreads, gemv_smem_bytes(2), s>>>(x, packed, alpha, y, int(M), N, K);
+  int C = 0, slice_words = 0, pages = 0;
+  if (M == 1 && lut_split(int(K), &C, &slice_words, &pages)) {
+    const bool overlap = (flags & BL_FLAG_OVERLAP_PREVIOUS) != 0;
+    cudaError_t e;
+    if (pages == 1)
+      e = launch_lut<1>(x, packed, alpha, y, int(N), int(K), C, slice_words, overlap, s);
+    else if (pages == 2)
+      e = launch_lut<2>(x, packed, alpha, y, int(N), int(K), C, slice_words, overlap, s);
     else
-      gemv_w1a16_kernel<4><<<grid, kGemvThreads, gemv_smem_bytes(4), s>>>(x, packed, alpha, y, int(M), N, K);
+      e = launch_lut<3>(x, packed, alpha, y, int(N), int(K), C, slice_words, overlap, s);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
     return launch_status();
   }
-  CUtensorMap tm_a, tm_bits;
-  if (!make_map_2d(&tm_a, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(K), uint64_t(M), 64, kBM,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4,
-                   GemmCfg<0>::BN, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return BL_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>(cdiv(N, GemmCfg<0>::BN)), static_cast<unsigned>(cdiv(M, kBM)));
-  gemm_bin_kernel<0><<<grid, kGemmThreads, GemmLayout<0>::SMEM_BYTES, s>>>(
-      tm_a, tm_bits, int(M), int(N), int(K), alpha, nullptr, nullptr, y, nullptr);
+  if (M > 4) {
+    int sms = 0;
+    device_setup(&sms);
+    if (M <= 32) return launch_ts<0, 32>(x, packed, M, N, K, alpha, nullptr, nullptr, y, nullptr, sms, s);
+    return launch_ts<0, 128>(x, packed, M, N, K, alpha, nullptr, nullptr, y, nullptr, sms, s);
+  }
+  const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
+  if (M == 1)
+    gemv_w1a16_kernel<1><<<grid, kGemvThreads, gemv_smem_bytes(1), s>>>(x, packed, alpha, y, int(M), N, K);
+  else if (M == 2)
+    gemv_w1a16_kernel<2><<<grid, kGemvThreads, gemv_smem_bytes(2), s>>>(x, packed, alpha, y, int(M), N, K);
+  else
+    gemv_w1a16_kernel<4><<<grid, kGemvThreads, gemv_smem_bytes(4), s>>>(x, packed, alpha, y, int(M), N, K);
   return launch_status();
 }
 

@@ -29,6 +29,7 @@ enum : int {
   kWhereGemmExpander = 2,
   kWhereGemmMma = 3,
   kWhereGemmEpilogue = 4,
+  kWhereLutInbox = 5,
 };
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.

@@ -100,11 +100,27 @@ int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, f
  *   y[m][j] = bf16( alpha[j] * sum_k s_jk * x[m][k] )
  * x [M x K] bf16, packed [N x K/32], alpha [N] fp32 (any values: the page
  * only initialises them), y [M x N] bf16 (round to nearest even).
- * Accumulation is fp32. Decode-sized M uses a bandwidth-bound GEMV kernel,
- * larger M a tcgen05 tensor-core GEMM. No workspace.
+ * Accumulation is fp32. A single token uses a lookup-table GEMV (a cluster
+ * of CTAs splits K; signed byte sums of x are tabulated in shared memory);
+ * up to 4 tokens a predicated-add GEMV; more tokens a tcgen05 tensor-core
+ * GEMM. No workspace.
  */
 int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
                      int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * bin_linear_w1a16_ex -- bin_linear_w1a16 with launch flags.
+ *   BL_FLAG_OVERLAP_PREVIOUS: the caller promises that `packed` and `alpha`
+ *   are not written by the kernel enqueued immediately before this call on
+ *   `stream` (true for a chain of inference layers). The single-token kernel
+ *   may then start streaming the weights before that kernel has finished
+ *   (programmatic dependent launch); it still waits for it before reading x
+ *   or writing y. Other kernels ignore the flag. flags = 0 is exactly
+ *   bin_linear_w1a16.
+ */
+#define BL_FLAG_OVERLAP_PREVIOUS 1u
+int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
+                        int64_t M, int64_t N, int64_t K, unsigned flags, void* stream);
 
 /*
  * bitlinear_w1a8 -- BitNet BitLinear forward ("BitNet b1.58" page,

@@ -36,8 +36,12 @@ def _to_dev(packed, alpha, x):
 
 
 FULL = [
-    # decode GEMV path (M <= 4)
-    (1, 128, 128), (1, 4096, 4096), (2, 300, 384), (3, 129, 256), (4, 1000, 11008), (1, 77, 8320),
+    # single-token lookup-table GEMV: cluster splits C=8 (1 and 3 pages), C=4, C=1, short rows,
+    # ragged row clusters, and K with no split (falls back to the predicated GEMV)
+    (1, 128, 128), (1, 4096, 4096), (1, 1000, 11008), (1, 257, 2048), (1, 300, 640), (1, 513, 5632),
+    (1, 4099, 384), (1, 77, 8320),
+    # few-token GEMV path (M <= 4)
+    (2, 300, 384), (3, 129, 256), (4, 1000, 11008),
     # tcgen05 GEMM path
     (5, 384, 256), (16, 128, 128), (17, 200, 384), (129, 383, 640), (256, 512, 1024),
     (300, 1000, 1024), (1000, 1100, 512),
@@ -130,3 +134,29 @@ def test_w1a16_negation_and_zero_tokens(bl):
     y0 = bl.bin_linear_w1a16(x[:0], packed, alpha)
     assert y0.shape == (0, N)
     torch.cuda.synchronize()
+
+
+def test_w1a16_overlap_flag_chain(bl, oracle):
+    """BL_FLAG_OVERLAP_PREVIOUS on a chain of dependent single-token calls
+    (each output is the next input): results must equal the oracle's."""
+    from bit_linear_layers_b200 import synthetic
+    N = K = 2048
+    layers = 6
+    Ws = [synthetic.weights(N, K, 100 + i) for i in range(layers)]
+    refs = [oracle.pack_fbi(W.numpy()) for W in Ws]
+    x = synthetic.activations(1, K, 7)
+    dev = [(torch.from_numpy(p.view(np.int32)).cuda(), torch.from_numpy(a).cuda()) for p, a in refs]
+    h = x.cuda()
+    outs = []
+    for (dp, da) in dev:
+        h = bl.bin_linear_w1a16(h, dp, da, flags=bl.BL_FLAG_OVERLAP_PREVIOUS)
+        outs.append(h)
+    torch.cuda.synchronize()
+    from bit_linear_layers_b200.synthetic import bf16_bits
+    xin = bf16_bits(x)
+    for i, ((p, a), y) in enumerate(zip(refs, outs)):
+        y_ref = oracle.w1a16(xin, p, a, K)
+        js = np.arange(N)
+        check_w1a16(bf16_to_f64(y).ravel(), y_ref.ravel(), a, xin, np.zeros(N, dtype=np.int64), js,
+                    what=f"layer {i}")
+        xin = bf16_bits(y.cpu())
