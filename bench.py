@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the prefill, W1A8 and 7B measurements that ride along at N=1")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -268,6 +270,174 @@ def cpu_baseline_decode(target_s=10.0, cap_s=30.0):
                       "(single-threaded C oracle, fp64)"}, np
 
 
+# ----------------------------------------------------------------------------- secondary
+
+def _flush_buffer(dev):
+    import torch
+    return torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MB > 126 MB L2
+
+
+def _timed_call(fn, flush, reps=5):
+    """Median device time (ms) of fn() with L2 flushed before every call."""
+    import torch
+    ts = []
+    for _ in range(2):
+        fn()
+    for _ in range(reps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    return ts[len(ts) // 2]
+
+
+def secondary_prefill(dev, peaks, flush):
+    """W1A16 prefill on the 7B MLP shapes: TFLOPS vs the measured bf16 peak."""
+    import bit_linear_layers_b200 as bl
+    from bit_linear_layers_b200 import synthetic
+    out, total_flop, total_ms = [], 0.0, 0.0
+    for (M, K, N) in [(2048, 4096, 11008), (2048, 11008, 4096)]:
+        W = synthetic.weights(N, K, seed=1, device=dev)
+        x = synthetic.activations(M, K, seed=1, device=dev)
+        p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
+        del W
+        ms = _timed_call(lambda: bl.bin_linear_w1a16(x, p, a), flush)
+        flop = 2.0 * M * N * K
+        out.append({"shape": f"{M}x{K}x{N}", "us": ms * 1e3, "tflops": flop / (ms * 1e-3) / 1e12})
+        total_flop += flop
+        total_ms += ms
+    tf = total_flop / (total_ms * 1e-3) / 1e12
+    return {"metric": "prefill TFLOPS (W1A16, 7B MLP shapes, 2048 tokens)", "tflops": tf,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / peaks["bf16_tflops"], "kernel": "gemm_ts_kernel<0,128>",
+                         "peak_source": "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops)"},
+            "shapes": out, "l2": "flushed (256 MB write) before every call"}
+
+
+def secondary_w1a8(dev, peaks, flush):
+    """BitLinear W1A8 at the 1.3B shapes (512 tokens): LN+quant and int8 GEMM."""
+    import torch
+    import bit_linear_layers_b200 as bl
+    from bit_linear_layers_b200 import synthetic
+    int8_peak = 2.0 * peaks["bf16_tflops"]
+    out, total_op, total_ms = [], 0.0, 0.0
+    for (M, K, N) in [(512, 2048, 5632), (512, 5632, 2048)]:
+        W = synthetic.weights(N, K, seed=4, mean=0.001, device=dev)
+        x = synthetic.laplace_channel_activations(M, K, seed=4, device=dev)
+        p, _, b = bl.bin_pack(W, bl.BL_PACK_BITNET)
+        del W
+        ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W1A8, M, N, K), dtype=torch.uint8, device=dev)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        ms = _timed_call(lambda: bl.bitlinear_w1a8(x, p, b, out=y, ws=ws), flush)
+        op = 2.0 * M * N * K
+        out.append({"shape": f"{M}x{K}x{N}", "us": ms * 1e3, "tops": op / (ms * 1e-3) / 1e12})
+        total_op += op
+        total_ms += ms
+    tops = total_op / (total_ms * 1e-3) / 1e12
+    return {"metric": "BitLinear W1A8 TOPS (1.3B shapes, 512 tokens, LN + quant + int8 GEMM)", "tops": tops,
+            "roofline": {"bound": "tensor", "achieved": tops, "peak": int8_peak, "unit": "TOP/s",
+                         "frac": tops / int8_peak,
+                         "peak_source": "measured bf16 burst x nominal int8/bf16 ratio 2"},
+            "shapes": out, "l2": "flushed (256 MB write) before every call"}
+
+
+def secondary_llama7b(dev, peaks):
+    """All 224 linears of a 7B-shaped model (0.8 GB of signs, more than L2):
+    decode at batch 1 and 16 as one dependent chain per token step
+    (x -> q,k,v; v -> o; o -> gate,up; up -> down -> next layer), CUDA graph
+    of one step, and a 4096-token prefill."""
+    import torch
+    import bit_linear_layers_b200 as bl
+    from bit_linear_layers_b200 import synthetic
+    layers = []
+    for layer in range(synthetic.LLAMA7B_LAYERS):
+        mats = []
+        for idx, (K, N) in enumerate(synthetic.LLAMA7B_LAYER):
+            W = synthetic.weights(N, K, seed=5000 + 16 * layer + idx, device=dev)
+            mats.append(bl.bin_pack(W, bl.BL_PACK_FBI))
+            del W
+        layers.append(mats)
+    packed_bytes = sum(p.numel() * 4 for mats in layers for p, _ in mats)
+    flags = bl.BL_FLAG_OVERLAP_PREVIOUS
+    res = {"packed_GB": packed_bytes / 1e9}
+    for B in (1, 16):
+        x = synthetic.activations(B, 4096, seed=77, device=dev)
+        bufs = {n: torch.empty((B, n), dtype=torch.bfloat16, device=dev) for n in (4096, 11008)}
+        q, k, v, o = (torch.empty((B, 4096), dtype=torch.bfloat16, device=dev) for _ in range(4))
+        g, u = (torch.empty((B, 11008), dtype=torch.bfloat16, device=dev) for _ in range(2))
+        h = torch.empty((B, 4096), dtype=torch.bfloat16, device=dev)
+
+        def step():
+            cur = x
+            for mats in layers:
+                bl.bin_linear_w1a16(cur, *mats[0], out=q, flags=flags)
+                bl.bin_linear_w1a16(cur, *mats[1], out=k, flags=flags)
+                bl.bin_linear_w1a16(cur, *mats[2], out=v, flags=flags)
+                bl.bin_linear_w1a16(v, *mats[3], out=o, flags=flags)
+                bl.bin_linear_w1a16(o, *mats[4], out=g, flags=flags)
+                bl.bin_linear_w1a16(o, *mats[5], out=u, flags=flags)
+                bl.bin_linear_w1a16(u, *mats[6], out=h, flags=flags)
+                cur = h
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        gph = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream(device=dev)
+        st.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(gph, stream=st):
+                step()
+        gph.replay()
+        torch.cuda.synchronize()
+        reps = 20
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            gph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[f"decode_batch{B}"] = {"ms_per_token_step": ms, "tok_s": B / (ms * 1e-3),
+                                   "packed_GB_per_s": packed_bytes / (ms * 1e-3) / 1e9,
+                                   "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                   "launches_per_step": 224}
+        del gph
+    # prefill: 4096 tokens through every linear (not chained: fixed inputs)
+    T = 4096
+    x4 = synthetic.activations(T, 4096, seed=78, device=dev)
+    x11 = synthetic.activations(T, 11008, seed=79, device=dev)
+    y4 = torch.empty((T, 4096), dtype=torch.bfloat16, device=dev)
+    y11 = torch.empty((T, 11008), dtype=torch.bfloat16, device=dev)
+
+    def prefill():
+        for mats in layers:
+            for idx, (K, N) in enumerate(synthetic.LLAMA7B_LAYER):
+                bl.bin_linear_w1a16(x4 if K == 4096 else x11, *mats[idx], out=y4 if N == 4096 else y11)
+
+    prefill()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    prefill()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    flop = sum(2.0 * T * K * N for (K, N) in synthetic.LLAMA7B_LAYER) * synthetic.LLAMA7B_LAYERS
+    res["prefill_4096"] = {"ms": ms, "tok_s": T / (ms * 1e-3), "tflops": flop / (ms * 1e-3) / 1e12,
+                           "tensor_frac": flop / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+                           "peak_source": "measured bf16 sustained (a long step)"}
+    res["metric"] = "linear-only tokens/s of a 7B-shaped FBI-LLM (32 layers x 7 linears)"
+    return res
+
+
 def bytes_per_step():
     packed = N_DEC * K_DEC // 8
     alg = packed + 4 * N_DEC + 2 * M_DEC * K_DEC + 2 * M_DEC * N_DEC
@@ -330,6 +500,15 @@ def main():
     value = world * args.steps * packed_b / (ms * 1e-3) / 1e9
     achieved = alg_b / (per_step_ms * 1e-3) / 1e9
     cpu, _ = cpu_baseline_decode()
+    secondary = None
+    if world == 1 and not args.no_secondary:
+        import torch
+        dev = torch.device("cuda", local_rank)
+        flush = _flush_buffer(dev)
+        secondary = {"prefill_w1a16": secondary_prefill(dev, peaks, flush),
+                     "w1a8_1p3b": secondary_w1a8(dev, peaks, flush)}
+        del flush
+        secondary["llama7b_linear"] = secondary_llama7b(dev, peaks)
     line = {
         "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
@@ -345,6 +524,7 @@ def main():
                 "ms_per_step": ms_e2e / args.steps},
         "gpu_launches": args.steps,
         "clocks": clocks,
+        "secondary": secondary,
     }
     print(json.dumps(line), flush=True)
     return 0
