@@ -42,6 +42,16 @@ bool set_smem(Kernel k, int bytes) {
   return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
+// every tensor-core GEMM configuration the dispatch below can launch
+template <int KIND>
+bool set_ts_smem() {
+  return set_smem(gemm_ts_kernel<KIND, 1, 256, false>, TsCfg<KIND, 1, 256, false>::SMEM_BYTES) &&
+         set_smem(gemm_ts_kernel<KIND, 2, 128, false>, TsCfg<KIND, 2, 128, false>::SMEM_BYTES) &&
+         set_smem(gemm_ts_kernel<KIND, 2, 128, true>, TsCfg<KIND, 2, 128, true>::SMEM_BYTES) &&
+         set_smem(gemm_ts_kernel<KIND, 2, 32, false>, TsCfg<KIND, 2, 32, false>::SMEM_BYTES) &&
+         set_smem(gemm_ts_kernel<KIND, 2, 32, true>, TsCfg<KIND, 2, 32, true>::SMEM_BYTES);
+}
+
 int device_setup(int* num_sms) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -63,10 +73,7 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<1>, 1 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<2>, 2 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
-              set_smem(gemm_ts_kernel<0, 32>, TsCfg<0, 32>::SMEM_BYTES) &&
-              set_smem(gemm_ts_kernel<0, 128>, TsCfg<0, 128>::SMEM_BYTES) &&
-              set_smem(gemm_ts_kernel<1, 32>, TsCfg<1, 32>::SMEM_BYTES) &&
-              set_smem(gemm_ts_kernel<1, 128>, TsCfg<1, 128>::SMEM_BYTES);
+              set_ts_smem<0>() && set_ts_smem<1>();
     if (!ok) cudaGetLastError();
     st.status = ok ? BL_OK : BL_ERR_CUDA;
   });
@@ -142,30 +149,94 @@ cudaError_t launch_lut(const uint16_t* x, const uint32_t* packed, const float* a
 
 // ---- tensor-core GEMM with the signs in tensor memory ------------------------------
 // activations [M][K] (bf16 for KIND 0, int8 codes for KIND 1) x packed signs [N][K/32]
-template <int KIND, int T>
-int launch_ts(const void* act, const uint32_t* packed, int64_t M, int64_t N, int64_t K,
-              const float* alpha, const double* gamma, const float* beta, void* y, int32_t* acc_out,
-              int num_sms, cudaStream_t s) {
-  using C = TsCfg<KIND, T>;
-  CUtensorMap tm_x, tm_bits;
-  const bool ok =
-      make_map_2d(&tm_x, act, KIND == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
-                  C::ELEM, uint64_t(K), uint64_t(M), 128 / C::ELEM, T, CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4,
-                  kTsRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (!ok) return BL_ERR_CUDA;
-  // output tile written by one bulk tensor store when the row pitch allows it
+// Split factor for a problem of `tiles` output tiles and `num_kb` k-blocks:
+// the largest S in {8, 4, 2} (S must divide the 256 rows of a tile) that
+// keeps tiles * S within the SMs and leaves every CTA at least one k-block.
+// Returns 1 when the persistent (unsplit) kernel should be used.
+int split_factor(int64_t tiles, int num_kb, int num_sms) {
+  for (int S : {8, 4, 2}) {
+    if (tiles * S > num_sms || S > num_kb) continue;
+    if (((num_kb + S - 1) / S) * (S - 1) >= num_kb) continue;
+    return S;
+  }
+  return 1;
+}
+
+template <int KIND, int NB, int T, bool SPLIT>
+int launch_ts_cfg(const CUtensorMap& tm_x, const CUtensorMap& tm_bits, int64_t M, int64_t N, int64_t K,
+                  int S, const float* alpha, const double* gamma, const float* beta, void* y,
+                  int32_t* acc_out, int num_sms, cudaStream_t s) {
+  using C = TsCfg<KIND, NB, T, SPLIT>;
+  const int64_t tiles = cdiv(M, T) * cdiv(N, C::ROWS);
   CUtensorMap tm_y;
   std::memset(&tm_y, 0, sizeof tm_y);
+  if (SPLIT) {
+    // a cluster of S CTAs per tile, each with a slice of the k-blocks
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(tiles), 1);
+    cfg.blockDim = dim3(kTsThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_ts_kernel<KIND, NB, T, SPLIT>, tm_x, tm_bits, tm_y, 0,
+                                             int(M), int(N), int(K), alpha, gamma, beta, y, acc_out);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    return launch_status();
+  }
+  // persistent: output tile written by one bulk tensor store when the row pitch allows it
   const int use_tma_store =
       (N * C::OUT_ELEM) % 16 == 0 &&
       make_map_2d(&tm_y, y, KIND == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                  C::OUT_ELEM, uint64_t(N), uint64_t(M), kTsRows, T, CU_TENSOR_MAP_SWIZZLE_NONE);
-  const int64_t tiles = cdiv(M, T) * cdiv(N, kTsRows);
+                  C::OUT_ELEM, uint64_t(N), uint64_t(M), C::ROWS, T, CU_TENSOR_MAP_SWIZZLE_NONE);
   const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
-  gemm_ts_kernel<KIND, T><<<grid, kTsThreads, C::SMEM_BYTES, s>>>(
+  gemm_ts_kernel<KIND, NB, T, SPLIT><<<grid, kTsThreads, C::SMEM_BYTES, s>>>(
       tm_x, tm_bits, tm_y, use_tma_store, int(M), int(N), int(K), alpha, gamma, beta, y, acc_out);
   return launch_status();
+}
+
+// activations [M][K] (bf16 for KIND 0, int8 codes for KIND 1) x packed signs [N][K/32].
+// Large bf16 problems: 128-row x 256-token tiles (one 128x256 MMA per K step),
+// persistent. Otherwise (and for int8, whose fp32 output tile would be too large
+// to stage for one bulk store) 256-row tiles of 128 or 32 tokens, split over a
+// cluster along K when the tiles alone would leave SMs idle.
+template <int KIND>
+int launch_ts(const void* act, const uint32_t* packed, int64_t M, int64_t N, int64_t K,
+              const float* alpha, const double* gamma, const float* beta, void* y, int32_t* acc_out,
+              int num_sms, cudaStream_t s) {
+  const int elem = KIND == 0 ? 2 : 1;
+  const CUtensorMapDataType xt = KIND == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const int num_kb = int(K / kTsStageK);
+  CUtensorMap tm_x, tm_bits;
+  const int64_t big_tiles = cdiv(M, 256) * cdiv(N, 128);
+  if (KIND == 0 && M >= 256 && 2 * big_tiles >= num_sms) {
+    if (!make_map_2d(&tm_x, act, xt, elem, uint64_t(K), uint64_t(M), 128 / elem, 256, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return BL_ERR_CUDA;
+    return launch_ts_cfg<KIND, 1, 256, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out,
+                                               num_sms, s);
+  }
+  const int T = M > 32 ? 128 : 32;
+  if (!make_map_2d(&tm_x, act, xt, elem, uint64_t(K), uint64_t(M), 128 / elem, uint32_t(T), CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4, 256,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BL_ERR_CUDA;
+  const int64_t tiles = cdiv(M, T) * cdiv(N, 256);
+  const int S = split_factor(tiles, num_kb, num_sms);
+  if (T == 128)
+    return S > 1 ? launch_ts_cfg<KIND, 2, 128, true>(tm_x, tm_bits, M, N, K, S, alpha, gamma, beta, y, acc_out, num_sms, s)
+                 : launch_ts_cfg<KIND, 2, 128, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out, num_sms, s);
+  return S > 1 ? launch_ts_cfg<KIND, 2, 32, true>(tm_x, tm_bits, M, N, K, S, alpha, gamma, beta, y, acc_out, num_sms, s)
+               : launch_ts_cfg<KIND, 2, 32, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out, num_sms, s);
 }
 
 // ---- W1A8 shared body -----------------------------------------------------------
@@ -215,9 +286,7 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
   }
   int sms = 0;
   device_setup(&sms);
-  if (M <= 32)
-    return launch_ts<1, 32>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s);
-  return launch_ts<1, 128>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s);
+  return launch_ts<1>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s);
 }
 
 }  // namespace
@@ -318,8 +387,7 @@ int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* 
   if (M > 4) {
     int sms = 0;
     device_setup(&sms);
-    if (M <= 32) return launch_ts<0, 32>(x, packed, M, N, K, alpha, nullptr, nullptr, y, nullptr, sms, s);
-    return launch_ts<0, 128>(x, packed, M, N, K, alpha, nullptr, nullptr, y, nullptr, sms, s);
+    return launch_ts<0>(x, packed, M, N, K, alpha, nullptr, nullptr, y, nullptr, sms, s);
   }
   const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
   if (M == 1)

@@ -8,21 +8,38 @@
 //     y[m][j]   = fp32( acc * beta * gamma_m / 128 )           fp64 epilogue
 //
 // The product is computed transposed, D[j][m] = sum_k S[j][k] X[m][k]: the
-// 1-bit weights are the MMA's M side (two M = 128 blocks per tile, 256 rows),
-// the tokens its N side (T per tile). Shared-memory traffic is then only the
+// 1-bit weights are the MMA's M side (NB blocks of 128 rows per tile), the
+// tokens its N side (T per tile). Shared-memory traffic is then only the
 // activation tile (TMA, 128-byte swizzle); the expanded +-1 signs never touch
 // shared memory: eight expander warps read each stage's packed bits, build
 // the +-1 operand in registers and write it to a ring of tensor-memory stages
-// with tcgen05.st. A tile moves T*2 + 256/8 bytes per k for 2*256*T flops.
+// with tcgen05.st.
+//
+// Each tcgen05.mma instruction costs the single issuing thread a roughly
+// fixed time, so the largest problems use 128 x 256 MMAs (NB = 1, T = 256):
+// enough tensor work per instruction to keep the pipe busy. Smaller problems
+// use two 128-row blocks (NB = 2) and fewer tokens per tile.
+//
+// The pipeline unit is one 128-byte swizzle atom of every activation row
+// (64 k for bf16, 128 k for int8). Activation units and 128-k sign stages
+// travel in separate shared-memory rings: the expanders only need the signs
+// and run ahead into a ring of tensor-memory sign units, while only the MMA
+// waits for the (much larger) activation units.
 //
 // Persistent kernel, one CTA per SM, 512 threads:
-//   warp 0      TMA producer: activation tile + packed sign tile per stage
+//   warp 0      TMA producer: sign stages and activation units
 //   warp 1      TMEM allocation; one thread issues the MMAs and commits
 //   warps 4..7  epilogue (tcgen05.ld of the accumulators, scale, store)
-//   warps 8..15 sign expanders: warp 8 + 4*b + q expands block b (rows
-//               128*b .. 128*b + 127) into TMEM lane quarter q = warp % 4
-// Tensor memory (512 columns): two accumulators of T columns, then the ring
-// of sign stages (two 128-row blocks per stage). All waits are bounded.
+//   warps 8..15 sign expanders; each writes one TMEM lane quarter (warp % 4)
+//               of one block (NB = 2) or of half a unit (NB = 1)
+// Tensor memory (512 columns): NB accumulators of T columns, then the ring
+// of sign units (NB blocks of 32 columns per unit). All waits are bounded.
+//
+// Split-K mode (few tiles, e.g. decode batches): a cluster of S CTAs shares
+// one tile and splits its k-blocks; each CTA pushes the partial sums of
+// every row to the CTA that owns the row (rows split S ways) with 16-byte
+// st.async stores counted on the owner's mbarrier, and the owner adds the S
+// partials in a fixed order (exact in int32 for W1A8) before the epilogue.
 #pragma once
 
 #include "bl_common.cuh"
@@ -31,34 +48,44 @@ namespace bl {
 
 constexpr int kTsThreads = 512;
 constexpr int kTsExpanders = 8;  // warps
-constexpr int kTsRows = 256;     // weight rows per tile (two UMMA M=128 blocks)
 constexpr int kTsStageK = 128;   // K elements per pipeline stage
 
-template <int KIND, int T>
+template <int KIND, int NB, int T, bool SPLIT>
 struct TsCfg {
+  static constexpr int ROWS = 128 * NB;                         // weight rows per tile
   static constexpr int ELEM = KIND == 0 ? 2 : 1;                // activation bytes
-  static constexpr int XSUB = kTsStageK * ELEM / 128;           // 128 B swizzle atoms per stage
-  static constexpr int X_SUB_BYTES = T * 128;
-  static constexpr int X_BYTES = X_SUB_BYTES * XSUB;
-  static constexpr int BITS_BYTES = kTsRows * 16;
-  static constexpr int STAGE_BYTES = X_BYTES + BITS_BYTES;
-  static constexpr int OUT_ELEM = KIND == 0 ? 2 : 4;             // y element bytes
-  static constexpr int OUT_BYTES = kTsRows * T * OUT_ELEM;         // staged output tile [T][256]
-  static constexpr int SX_FIT = (208 * 1024 - OUT_BYTES) / STAGE_BYTES;
-  static constexpr int SX = SX_FIT > 8 ? 8 : SX_FIT;
-  static constexpr int SMEM_BYTES = SX * STAGE_BYTES + OUT_BYTES + 1024;
+  // pipeline unit: one 128-byte swizzle atom of every activation row
+  static constexpr int UNIT_K = 128 / ELEM;                     // 64 (bf16) or 128 (int8)
+  static constexpr int UPB = ELEM;                              // units per 128-k sign stage
+  static constexpr int X_UNIT_BYTES = T * 128;
+  static constexpr int BITS_BYTES = ROWS * 16;                  // one 128-k sign stage
+  static constexpr int SB = 4;                                  // sign stages in shared memory
+  static constexpr int OUT_ELEM = KIND == 0 ? 2 : 4;            // y element bytes
+  // the output tile is staged for one bulk store when it fits in 64 KB
+  static constexpr bool STAGE_OUT = !SPLIT && ROWS * T * OUT_ELEM <= 64 * 1024;
+  // staged output tile [T][ROWS], or the split-K inbox of 4-byte partials [S][ROWS/S][T]
+  static constexpr int OUT_BYTES = SPLIT ? ROWS * T * 4 : (STAGE_OUT ? ROWS * T * OUT_ELEM : 0);
+  static constexpr int SX_FIT = (210 * 1024 - OUT_BYTES - SB * BITS_BYTES) / X_UNIT_BYTES;
+  static constexpr int SX = SX_FIT > 8 ? 8 : SX_FIT;           // activation units in flight
+  static constexpr int X_RING = SX * X_UNIT_BYTES;
+  static constexpr int SMEM_BYTES = X_RING + SB * BITS_BYTES + OUT_BYTES + 1024;
   static constexpr int MMA_K = KIND == 0 ? 16 : 32;             // elements per MMA
-  static constexpr int KSTEPS = kTsStageK / MMA_K;              // MMAs per block per stage
-  static constexpr int A_COLS = kTsStageK * ELEM / 4;           // TMEM columns per block per stage
-  static constexpr int D_COLS = 2 * T;                          // two accumulators
-  static constexpr int SA_MAX = (512 - D_COLS) / (2 * A_COLS);
-  static constexpr int SA = SA_MAX > 4 ? 4 : SA_MAX;            // sign stages in TMEM
-  static_assert(SA >= 2, "need at least two sign stages");
-  static_assert(SX >= 2, "need at least two activation stages");
-  static_assert(X_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle alignment");
+  static constexpr int KSTEPS = 4;                              // MMAs per block per unit (32 B each)
+  static constexpr int A_COLS = 32;                             // TMEM columns per block per unit
+  static constexpr int CH = UNIT_K / 16;                        // 16-bit sign chunks per unit
+  static constexpr int D_COLS = NB * T;                         // accumulators
+  static constexpr int SA_MAX = (512 - D_COLS) / (NB * A_COLS);
+  static constexpr int SA = SA_MAX > 8 ? 8 : SA_MAX;            // sign units in TMEM
+  static_assert(SA >= 2, "need at least two sign units");
+  static_assert(SX >= 2, "need at least two activation units");
+  static_assert(X_UNIT_BYTES % 1024 == 0 && BITS_BYTES % 1024 == 0, "swizzle alignment");
+  static_assert(NB == 1 || NB == 2, "one or two 128-row blocks per tile");
 };
 
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+template <int N>
+__device__ __forceinline__ void tmem_st_32x32b(uint32_t taddr, const uint32_t* r);
+template <>
+__device__ __forceinline__ void tmem_st_32x32b<32>(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
@@ -67,6 +94,15 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_st_32x32b<16>(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -118,31 +154,65 @@ __device__ __forceinline__ void expand16_i8(uint32_t bits, uint32_t* out) {
   }
 }
 
-template <int KIND, int T>
+__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, const uint32_t* v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   remote_addr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(remote_bar)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t ts_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t ts_map_rank(uint32_t local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  return remote;
+}
+
+template <int KIND, int NB, int T, bool SPLIT>
 __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_bits,
     const __grid_constant__ CUtensorMap tm_y, int use_tma_store, int M, int N, int K,
     const float* __restrict__ alpha, const double* __restrict__ gamma, const float* __restrict__ beta,
     void* __restrict__ y, int32_t* __restrict__ acc_out) {
-  using C = TsCfg<KIND, T>;
-  constexpr int SX = C::SX, SA = C::SA;
+  using C = TsCfg<KIND, NB, T, SPLIT>;
+  constexpr int SX = C::SX, SA = C::SA, ROWS = C::ROWS;
 
   extern __shared__ uint8_t ts_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ts_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t x_full[SX], x_empty[SX], a_full[SA], a_empty[SA], d_full, d_empty;
+  __shared__ __align__(8) uint64_t x_full[SX], x_empty[SX], b_full[C::SB], b_empty[C::SB];
+  __shared__ __align__(8) uint64_t a_full[SA], a_empty[SA], d_full, d_empty;
   __shared__ uint32_t tmem_base_sh;
+  __shared__ __align__(8) uint64_t inbox_bar;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_kb = K / kTsStageK;
   const int tiles_t = (M + T - 1) / T;
-  const int tiles_w = (N + kTsRows - 1) / kTsRows;
+  const int tiles_w = (N + ROWS - 1) / ROWS;
   const int num_tiles = tiles_t * tiles_w;
+  // persistent over tiles; in split-K mode one tile per cluster and a k range per CTA
+  const int tile_first = SPLIT ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
+  const int tile_step = SPLIT ? static_cast<int>(gridDim.y) : static_cast<int>(gridDim.x);
+  const uint32_t rank = SPLIT ? ts_cluster_rank() : 0u;
+  const int S = SPLIT ? static_cast<int>(gridDim.x) : 1;
+  const int kb_per = (num_kb + S - 1) / S;
+  const int kb_first = SPLIT ? static_cast<int>(rank) * kb_per : 0;
+  const int kb_last = SPLIT ? min(num_kb, kb_first + kb_per) : num_kb;
+  // pipeline units of this CTA within each tile (whole sign stages)
+  const int u_first = kb_first * C::UPB, u_last = kb_last * C::UPB;
+  uint8_t* const bits_ring = smem + C::X_RING;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; ++s) {
       mbar_init(smem_u32(&x_full[s]), 1);
-      mbar_init(smem_u32(&x_empty[s]), 1 + kTsExpanders);  // MMA commit + expander warps
+      mbar_init(smem_u32(&x_empty[s]), 1);  // MMA commit
+    }
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(smem_u32(&b_full[s]), 1);
+      mbar_init(smem_u32(&b_empty[s]), kTsExpanders);
     }
     for (int a = 0; a < SA; ++a) {
       mbar_init(smem_u32(&a_full[a]), kTsExpanders);
@@ -150,6 +220,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     }
     mbar_init(smem_u32(&d_full), 1);
     mbar_init(smem_u32(&d_empty), 4);
+    if (SPLIT) mbar_init(smem_u32(&inbox_bar), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_bits);
@@ -162,29 +233,39 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  if (SPLIT) asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");  // waited before pushing
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t a_base = tmem + C::D_COLS;  // sign ring starts after the two accumulators
+  const uint32_t a_base = tmem + C::D_COLS;  // sign ring starts after the accumulators
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
+    // per unit: the sign stage (every UPB units) first, the expanders need
+    // only those; then the activation atom the MMA reads
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * kTsRows;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const uint32_t s = it % SX;
-          if (it >= SX && !mbar_wait(smem_u32(&x_empty[s]), ((it / SX) - 1) & 1, kWhereGemmProducer)) {
+      for (int tile = tile_first; tile < num_tiles && ok; tile += tile_step) {
+        const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
+        for (int u = u_first; u < u_last; ++u, ++it) {
+          if (it % C::UPB == 0) {
+            const uint32_t bit_it = it / C::UPB, bs = bit_it % C::SB;
+            if (bit_it >= C::SB &&
+                !mbar_wait(smem_u32(&b_empty[bs]), ((bit_it / C::SB) - 1) & 1, kWhereGemmProducer)) {
+              ok = false;
+              break;
+            }
+            const uint32_t bb = smem_u32(&b_full[bs]);
+            mbar_arrive_expect_tx(bb, C::BITS_BYTES);
+            tma_load_2d(smem_u32(bits_ring + bs * C::BITS_BYTES), &tm_bits, bb, (u / C::UPB) * 4, w0);
+          }
+          const uint32_t xs = it % SX;
+          if (it >= SX && !mbar_wait(smem_u32(&x_empty[xs]), ((it / SX) - 1) & 1, kWhereGemmProducer)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * C::STAGE_BYTES;
-          const uint32_t fb = smem_u32(&x_full[s]);
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-#pragma unroll
-          for (int h = 0; h < C::XSUB; ++h)
-            tma_load_2d(smem_u32(st + h * C::X_SUB_BYTES), &tm_x, fb, kb * kTsStageK + h * (128 / C::ELEM), t0);
-          tma_load_2d(smem_u32(st + C::X_BYTES), &tm_bits, fb, kb * (kTsStageK / 32), w0);
+          const uint32_t fb = smem_u32(&x_full[xs]);
+          mbar_arrive_expect_tx(fb, C::X_UNIT_BYTES);
+          tma_load_2d(smem_u32(smem + xs * C::X_UNIT_BYTES), &tm_x, fb, u * C::UNIT_K, t0);
         }
       }
     }
@@ -194,35 +275,36 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
       const uint32_t idesc = KIND == 0 ? idesc_bf16_f32(128, T) : idesc_s8_s32(128, T);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
+      for (int tile = tile_first; tile < num_tiles && ok; tile += tile_step, ++tcount) {
         if (tcount > 0 && !mbar_wait(smem_u32(&d_empty), (tcount - 1) & 1, kWhereGemmMma)) break;
         tc_fence_after_sync();
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const uint32_t s = it % SX, a = it % SA;
-          if (!mbar_wait(smem_u32(&x_full[s]), (it / SX) & 1, kWhereGemmMma) ||
+        for (int u = u_first; u < u_last; ++u, ++it) {
+          const uint32_t xs = it % SX, a = it % SA;
+          if (!mbar_wait(smem_u32(&x_full[xs]), (it / SX) & 1, kWhereGemmMma) ||
               !mbar_wait(smem_u32(&a_full[a]), (it / SA) & 1, kWhereGemmMma)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t xs = smem_u32(smem + s * C::STAGE_BYTES);
+          // descriptor of the atom's first 32-byte K slice; later slices add
+          // their byte offset >> 4 to the start-address field (never carries:
+          // the ring lies inside the 256 KB window of the 14-bit field)
+          const uint64_t bd0 = sw128_kmajor_desc(smem_u32(smem + xs * C::X_UNIT_BYTES));
+          const uint32_t a_tm0 = a_base + (a * NB) * C::A_COLS;
 #pragma unroll
-          for (int blk = 0; blk < 2; ++blk) {
-            const uint32_t a_tm = a_base + (a * 2 + blk) * C::A_COLS;
-            const uint32_t d_tm = tmem + blk * T;
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint64_t bd = bd0 + static_cast<uint64_t>((kk * 32) >> 4);
+            const uint32_t accum = (u > u_first || kk > 0) ? 1u : 0u;
 #pragma unroll
-            for (int kk = 0; kk < C::KSTEPS; ++kk) {
-              // MMA_K elements = 32 bytes of an activation row; 4 per 128-byte atom
-              const uint32_t xaddr = xs + (kk / 4) * C::X_SUB_BYTES + (kk % 4) * 32;
-              const uint64_t bd = sw128_kmajor_desc(xaddr);
-              const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            for (int blk = 0; blk < NB; ++blk) {
+              const uint32_t a_tm = a_tm0 + blk * C::A_COLS + kk * 8;
               if (KIND == 0)
-                umma_ts_bf16(d_tm, a_tm + kk * 8, bd, idesc, accum);
+                umma_ts_bf16(tmem + blk * T, a_tm, bd, idesc, accum);
               else
-                umma_ts_i8(d_tm, a_tm + kk * 8, bd, idesc, accum);
+                umma_ts_i8(tmem + blk * T, a_tm, bd, idesc, accum);
             }
           }
-          umma_commit(smem_u32(&x_empty[s]));
+          umma_commit(smem_u32(&x_empty[xs]));
           umma_commit(smem_u32(&a_empty[a]));
         }
         if (!ok) break;
@@ -231,72 +313,138 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     }
   } else if (warp >= 8) {
     // ---------------- sign expanders ----------------
-    const int q = warp & 3, blk = (warp - 8) >> 2;
+    // With two blocks, warp 8 + 4*b + q expands block b, lane quarter q, all
+    // CH chunks of the unit; with one block the two warps of a lane quarter
+    // take half of the chunks each. A unit's signs are 16-bit chunks
+    // g = h*CH + j of the 128-bit stage row (h = unit within the stage).
+    const int q = warp & 3, part = (warp - 8) >> 2;
+    const int blk = NB == 2 ? part : 0;
+    constexpr int MY_CH = NB == 2 ? C::CH : C::CH / 2;      // chunks this warp expands
+    constexpr int COLS_PER_CH = C::A_COLS / C::CH;           // 8 (bf16) or 4 (int8)
+    const int ch0 = NB == 2 ? 0 : part * MY_CH;
     const int r = blk * 128 + q * 32 + lane;  // sign row within the tile = TMEM lane in its block
     uint32_t it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
-        const uint32_t s = it % SX, a = it % SA;
-        if (!mbar_wait(smem_u32(&x_full[s]), (it / SX) & 1, kWhereGemmExpander) ||
-            (it >= SA && !mbar_wait(smem_u32(&a_empty[a]), ((it / SA) - 1) & 1, kWhereGemmExpander))) {
+    for (int tile = tile_first; tile < num_tiles && ok; tile += tile_step) {
+      for (int u = u_first; u < u_last; ++u, ++it) {
+        const uint32_t a = it % SA, bit_it = it / C::UPB, bs = bit_it % C::SB;
+        if ((it >= SA && !mbar_wait(smem_u32(&a_empty[a]), ((it / SA) - 1) & 1, kWhereGemmExpander)) ||
+            !mbar_wait(smem_u32(&b_full[bs]), (bit_it / C::SB) & 1, kWhereGemmExpander)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint8_t* bits = smem + s * C::STAGE_BYTES + C::X_BYTES;
-        const uint4 wv = *reinterpret_cast<const uint4*>(bits + r * 16);
+        const uint4 wv = *reinterpret_cast<const uint4*>(bits_ring + bs * C::BITS_BYTES + r * 16);
         const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-        const uint32_t taddr = a_base + (a * 2 + blk) * C::A_COLS + (static_cast<uint32_t>(q * 32) << 16);
-        if (KIND == 0) {
-          // 128 bf16 = 64 columns, written as two halves of 32
+        const int h = static_cast<int>(it % C::UPB);
+        const uint32_t taddr = a_base + (a * NB + blk) * C::A_COLS + ch0 * COLS_PER_CH +
+                               (static_cast<uint32_t>(q * 32) << 16);
+        // this warp's chunks are words off_w .. off_w + MY_CH/2 - 1 of the row
+        constexpr int MY_W = MY_CH / 2;
+        const int off_w = (h * C::CH + ch0) >> 1;  // even chunk offset
+        uint32_t seg[MY_W];
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              expand16_bf16((wd[half * 2 + j / 2] >> (16 * (j & 1))) & 0xFFFFu, v + 8 * j);
-            tmem_st_32x32b_x32(taddr + half * 32, v);
-          }
-        } else {
-          // 128 int8 = 32 columns
-          uint32_t v[32];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) expand16_i8((wd[j / 2] >> (16 * (j & 1))) & 0xFFFFu, v + 4 * j);
-          tmem_st_32x32b_x32(taddr, v);
+        for (int w = 0; w < MY_W; ++w) {
+          const int idx = off_w + w;
+          seg[w] = idx == 0 ? wd[0] : idx == 1 ? wd[1] : idx == 2 ? wd[2] : wd[3];
         }
+        uint32_t v[MY_CH * COLS_PER_CH];
+#pragma unroll
+        for (int j = 0; j < MY_CH; ++j) {
+          const uint32_t chunk = (seg[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+          if (KIND == 0)
+            expand16_bf16(chunk, v + j * COLS_PER_CH);
+          else
+            expand16_i8(chunk, v + j * COLS_PER_CH);
+        }
+        tmem_st_32x32b<MY_CH * COLS_PER_CH>(taddr, v);
         tmem_wait_st();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(smem_u32(&a_full[a]));
-          mbar_arrive(smem_u32(&x_empty[s]));
+          if (it % C::UPB == C::UPB - 1) mbar_arrive(smem_u32(&b_empty[bs]));
+        }
+      }
+    }
+  } else if (warp >= 4 && SPLIT) {
+    // ---------------- split-K epilogue: push partials, owner reduces ----------------
+    const int q = warp & 3;
+    const int rows_per = ROWS / S;                      // rows owned by each CTA of the cluster
+    uint8_t* inbox = bits_ring + C::SB * C::BITS_BYTES;  // [S][rows_per][T] 4-byte partials
+    const int tile = tile_first;
+    const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
+    bool ok = true;
+    if (threadIdx.x == 128) mbar_arrive_expect_tx(smem_u32(&inbox_bar), ROWS * T * 4);
+    asm volatile("barrier.cluster.wait;" ::: "memory");  // every inbox barrier is initialised
+    if (!mbar_wait(smem_u32(&d_full), 0, kWhereGemmEpilogue)) ok = false;
+    tc_fence_after_sync();
+#pragma unroll 1
+    for (int blk = 0; blk < NB && ok; ++blk) {
+      const int jl = blk * 128 + q * 32 + lane;
+      const uint32_t owner = static_cast<uint32_t>(jl / rows_per);
+      const uint32_t slot0 =
+          smem_u32(inbox + (static_cast<int>(rank) * rows_per + jl % rows_per) * T * 4);
+      const uint32_t rslot = ts_map_rank(slot0, owner);
+      const uint32_t rbar = ts_map_rank(smem_u32(&inbox_bar), owner);
+#pragma unroll 1
+      for (int cc = 0; cc < T / 32; ++cc) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem + blk * T + cc * 32 + (static_cast<uint32_t>(q * 32) << 16), r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int v = 0; v < 8; ++v) st_async_v4(rslot + (cc * 32 + v * 4) * 4, r + v * 4, rbar);
+      }
+    }
+    // owner: add the S partials of its rows in rank order, then scale and store
+    if (ok && mbar_wait(smem_u32(&inbox_bar), 0, kWhereGemmEpilogue)) {
+      const int et = threadIdx.x - 128;  // 0..127
+      double bt = 0.0;
+      if (KIND == 1) bt = static_cast<double>(*beta);
+      for (int e = et; e < rows_per * T; e += 128) {
+        const int rr = e % rows_per, tt = e / rows_per;
+        const int j = w0 + static_cast<int>(rank) * rows_per + rr, m = t0 + tt;
+        if (j >= N || m >= M) continue;
+        const int64_t o = static_cast<int64_t>(m) * N + j;
+        if (KIND == 0) {
+          float acc = 0.f;
+          for (int src = 0; src < S; ++src)
+            acc += reinterpret_cast<const float*>(inbox)[(src * rows_per + rr) * T + tt];
+          reinterpret_cast<uint16_t*>(y)[o] = float_to_bf16_bits(acc * alpha[j]);
+        } else {
+          int32_t acc = 0;
+          for (int src = 0; src < S; ++src)
+            acc += reinterpret_cast<const int32_t*>(inbox)[(src * rows_per + rr) * T + tt];
+          reinterpret_cast<float*>(y)[o] = static_cast<float>(static_cast<double>(acc) * bt * gamma[m] / 128.0);
+          if (acc_out) acc_out[o] = acc;
         }
       }
     }
   } else if (warp >= 4) {
     // ---------------- epilogue ----------------
-    // Accumulators -> scaled outputs -> staging tile [T tokens][256 rows] in
+    // Accumulators -> scaled outputs -> staging tile [T tokens][ROWS] in
     // shared memory; the accumulators are released as soon as they are read,
     // then one bulk tensor store writes the tile (rows/tokens past N/M are
     // clipped by the store). Without an aligned output (N % 8 for bf16,
-    // N % 4 for fp32) the outputs are stored directly instead.
+    // N % 4 for fp32), or when the tile is too large to stage, the outputs
+    // are stored directly instead.
     const int q = warp & 3;
-    uint8_t* stage_out = smem + SX * C::STAGE_BYTES;
+    uint8_t* stage_out = bits_ring + C::SB * C::BITS_BYTES;
     const bool leader = (warp == 4 && lane == 0);
     uint32_t tcount = 0;
     double bt = 0.0;
     if (KIND == 1) bt = static_cast<double>(*beta);
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
-      const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * kTsRows;
+    for (int tile = tile_first; tile < num_tiles; tile += tile_step, ++tcount) {
+      const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
       if (!mbar_wait(smem_u32(&d_full), tcount & 1, kWhereGemmEpilogue)) break;
       tc_fence_after_sync();
-      if (use_tma_store) {
+      if (C::STAGE_OUT && use_tma_store) {
         if (leader) bulk_wait_read0();  // the previous tile's store has read the staging tile
         epilogue_bar();
       }
 #pragma unroll 1
-      for (int blk = 0; blk < 2; ++blk) {
+      for (int blk = 0; blk < NB; ++blk) {
         const int jl = blk * 128 + q * 32 + lane;  // row of the tile = output channel w0 + jl
         const int j = w0 + jl;
         const bool jv = j < N;
@@ -308,7 +456,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
           __syncwarp();
           tmem_ld_32x32b_x32(tmem + blk * T + cc * 32 + (static_cast<uint32_t>(q * 32) << 16), r);
           tmem_wait_ld();
-          if (blk == 1 && cc == T / 32 - 1) {
+          if (blk == NB - 1 && cc == T / 32 - 1) {
             // every accumulator column of this tile has been read: free them
             tc_fence_before_sync();
             __syncwarp();
@@ -320,16 +468,16 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
             const int m = t0 + ml0 + i;
             if (KIND == 0) {
               const uint16_t v = float_to_bf16_bits(__uint_as_float(r[i]) * aj);
-              if (use_tma_store)
-                reinterpret_cast<uint16_t*>(stage_out)[(ml0 + i) * kTsRows + jl] = v;
+              if (C::STAGE_OUT && use_tma_store)
+                reinterpret_cast<uint16_t*>(stage_out)[(ml0 + i) * ROWS + jl] = v;
               else if (jv && m < M)
                 reinterpret_cast<uint16_t*>(y)[static_cast<int64_t>(m) * N + j] = v;
             } else {
               const int32_t acc = static_cast<int32_t>(r[i]);
               const double gm = m < M ? gamma[m] : 0.0;
               const float v = static_cast<float>(static_cast<double>(acc) * bt * gm / 128.0);
-              if (use_tma_store)
-                reinterpret_cast<float*>(stage_out)[(ml0 + i) * kTsRows + jl] = v;
+              if (C::STAGE_OUT && use_tma_store)
+                reinterpret_cast<float*>(stage_out)[(ml0 + i) * ROWS + jl] = v;
               else if (jv && m < M)
                 reinterpret_cast<float*>(y)[static_cast<int64_t>(m) * N + j] = v;
               if (acc_out && jv && m < M) acc_out[static_cast<int64_t>(m) * N + j] = acc;
@@ -337,7 +485,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
           }
         }
       }
-      if (use_tma_store) {
+      if (C::STAGE_OUT && use_tma_store) {
         fence_proxy_async_smem();  // staging writes -> visible to the bulk store
         epilogue_bar();
         if (leader) {
@@ -346,9 +494,11 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
         }
       }
     }
-    if (use_tma_store && leader) bulk_wait0();
+    if (C::STAGE_OUT && use_tma_store && leader) bulk_wait0();
   }
 
+  if (SPLIT && !(warp >= 4 && warp < 8))
+    asm volatile("barrier.cluster.wait;" ::: "memory");  // matches the arrive above (lanes may diverge)
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 1) {

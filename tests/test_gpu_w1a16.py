@@ -45,6 +45,8 @@ FULL = [
     # tcgen05 GEMM path
     (5, 384, 256), (16, 128, 128), (17, 200, 384), (129, 383, 640), (256, 512, 1024),
     (300, 1000, 1024), (1000, 1100, 512),
+    # enough tiles for the 128-row x 256-token configuration, ragged in M and N
+    (300, 9100, 256),
 ]
 
 
