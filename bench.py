@@ -2,25 +2,35 @@
 """Benchmark of the binarized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill|w1a8] [--no-secondary]
 
-Default workload: the FBI-linear W1A16 decode GEMV, M=1 token, K=N=4096
-(a 7B attention projection), judged on packed-weight bytes per second. A
-step is one call of the layer on one token. Between steps the weights
-rotate over 128 distinct packed copies (268 MB, more than twice the 126 MB
-L2), so every step streams its weights from HBM. After W untimed warm-up
-steps, K steps are captured in one CUDA graph and timed with CUDA events on
-the launching stream; with N ranks (torchrun) every rank runs its own
-replica (no data-path collective) and the time is the max over ranks.
+Workloads (a step is one pass of the layer over one batch of synthetic input):
 
-Rank 0 prints one JSON line. `--impl reference` times the CPU oracle on the
-same workload instead (the reference arm of this benchmark).
+* ``decode`` (default, the headline): FBI-linear W1A16 GEMV, M=1 token,
+  K=N=4096 (a 7B attention projection), judged on packed-weight bytes per
+  second against the measured HBM bandwidth;
+* ``prefill``: FBI-linear W1A16 on the 7B MLP shapes, 2048 tokens, the
+  up-projection 4096->11008 then the down-projection 11008->4096, judged in
+  TFLOP/s against the measured bf16 tensor peak;
+* ``w1a8``: BitNet BitLinear (LN + absmax int8 quantisation + int8 GEMM +
+  rescale) on the 1.3B shapes, 512 tokens, 2048->5632 then 5632->2048, in
+  TOP/s against the int8 tensor peak.
+
+Each workload keeps R distinct copies of its weights and activations whose
+total is more than twice the 126 MB L2, and step i uses copy i % R, so no step
+finds its inputs in L2. After W untimed warm-up steps, K steps are captured
+in one CUDA graph and timed with CUDA events on the launching stream; with N
+ranks (torchrun) every rank runs its own replica (no data-path collective)
+and the time is the max over ranks.
+
+Rank 0 prints one JSON line. `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead (the reference arm).
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -33,11 +43,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-M_DEC, K_DEC, N_DEC = 1, 4096, 4096
-ROTATE = 128
-KERNEL_SOURCES = ["bit_linear_layers_b200/csrc/bl_gemv_lut.cuh", "bit_linear_layers_b200/csrc/bl_common.cuh",
-                  "bit_linear_layers_b200/csrc/bl_api.cu"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_w1a16_decode_1x4096x4096.traffic.json")
+CSRC = "bit_linear_layers_b200/csrc/"
+SUSTAINED_AFTER_S = 1.0  # a timed region longer than this runs under the power cap: sustained peak
 
 
 def parse():
@@ -46,8 +53,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the prefill, W1A8 and 7B measurements that ride along at N=1")
+                    help="skip the other workloads and the 7B measurement that ride along at N=1")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -63,24 +71,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_src_hash() -> str:
+def src_hash(sources) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
-
-
-def traffic_per_launch():
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    summary is missing or was taken on a different version of the kernel."""
-    if not os.path.exists(TRAFFIC_FILE):
-        return None
-    with open(TRAFFIC_FILE) as f:
-        d = json.load(f)
-    if d.get("src_hash") != kernel_src_hash():
-        return None
-    return d.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
@@ -133,68 +129,321 @@ class ClockSampler:
                 "samples": len(sm), "window": "warm-up and timed steps"}
 
 
+# ----------------------------------------------------------------------------- workloads
+
+
+class Workload:
+    """One benchmarked configuration: its rotating device copies, a device
+    step, an end-to-end step through pinned host buffers, and the oracle's
+    bounded sample of the same work."""
+
+    name = ""
+    metric = ""
+    unit = ""
+    scale = 1e9          # unit = work units per second / scale
+    dtype = "bf16"
+    bound = "hbm"
+    kernel = ""
+    sources: list = []
+    traffic_file = None
+    launches_per_step = 1
+    rotate = 1
+    config: dict = {}
+
+    def units_per_step(self) -> float:
+        raise NotImplementedError
+
+    def achieved(self, per_step_s: float) -> float:
+        """Algorithmic bytes (or flops) of the dominant kernel per launch over its launch time."""
+        return self.units_per_step() / per_step_s / self.scale
+
+    def peak(self, peaks, timed_s):
+        raise NotImplementedError
+
+    def traffic(self):
+        """DRAM bytes per launch from the committed ncu summary, or None when
+        the summary is missing or was taken on another version of the kernel."""
+        if self.traffic_file is None:
+            return None
+        path = os.path.join(ROOT, "profiles", self.traffic_file)
+        if not os.path.exists(path):
+            return None
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("src_hash") != src_hash(self.sources):
+            return None
+        return d.get("dram_bytes_per_launch")
+
+
+class Decode(Workload):
+    name = "decode"
+    M, K, N = 1, 4096, 4096
+    metric = "decode GEMV HBM GB/s on packed-weight bytes (W1A16, 1x4096x4096)"
+    unit, scale, bound = "GB/s", 1e9, "hbm"
+    kernel = "gemv_w1a16_lut_kernel<1> (cluster of 8 x 16 clusters)"
+    sources = [CSRC + "bl_gemv_lut.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = "gemv_w1a16_decode_1x4096x4096.traffic.json"
+    rotate = 128
+
+    def __init__(self):
+        self.packed_b = self.N * self.K // 8
+        self.alg_b = self.packed_b + 4 * self.N + 2 * self.M * self.K + 2 * self.M * self.N
+        self.config = {"workload": "FBI-linear W1A16 decode GEMV, M=1, K=4096, N=4096 (7B attention projection)",
+                       "M": self.M, "K": self.K, "N": self.N,
+                       "l2": f"inputs larger than L2: {self.rotate} distinct packed weight copies "
+                             f"({self.rotate * self.packed_b / 1e6:.0f} MB) rotated step to step",
+                       "launch": "programmatic dependent launch between steps (BL_FLAG_OVERLAP_PREVIOUS)"}
+
+    def units_per_step(self):
+        return self.packed_b  # the metric counts packed-weight bytes
+
+    def achieved(self, per_step_s):
+        return self.alg_b / per_step_s / 1e9  # all bytes the kernel must move
+
+    def peak(self, peaks, timed_s):
+        return peaks["hbm_gbs"], "hbm_gbs"
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        from bit_linear_layers_b200 import synthetic
+        self.bl = bl
+        self.packs, self.alphas, self.xs = [], [], []
+        for i in range(self.rotate):
+            if i == 0:  # the seeded workload itself (CPU generator)
+                W = synthetic.weights(self.N, self.K, seed=2).to(dev)
+                x = synthetic.activations(self.M, self.K, seed=2).to(dev)
+            else:       # further seeded draws made on the device
+                W = synthetic.weights(self.N, self.K, seed=2 + 1000 * i + 7 * rank, device=dev)
+                x = synthetic.activations(self.M, self.K, seed=2 + 1000 * i + 7 * rank, device=dev)
+            p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
+            self.packs.append(p)
+            self.alphas.append(a)
+            self.xs.append(x)
+            del W
+        self.ys = [torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev) for _ in range(self.rotate)]
+        # consecutive steps never write each other's inputs, so each launch may
+        # start streaming its weights while the previous one finishes
+        self.flags = bl.BL_FLAG_OVERLAP_PREVIOUS
+        self.xh = [x.cpu().pin_memory() for x in self.xs]
+        self.yh = [torch.empty((self.M, self.N), dtype=torch.bfloat16).pin_memory() for _ in range(self.rotate)]
+        self.xd = torch.empty((self.M, self.K), dtype=torch.bfloat16, device=dev)
+        self.yd = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        self.h2d, self.d2h = 2 * self.M * self.K, 2 * self.M * self.N
+
+    def step(self, i):
+        j = i % self.rotate
+        self.bl.bin_linear_w1a16(self.xs[j], self.packs[j], self.alphas[j], out=self.ys[j], flags=self.flags)
+
+    def e2e_step(self, i):
+        j = i % self.rotate
+        self.xd.copy_(self.xh[j], non_blocking=True)
+        self.bl.bin_linear_w1a16(self.xd, self.packs[j], self.alphas[j], out=self.yd, flags=self.flags)
+        self.yh[j].copy_(self.yd, non_blocking=True)
+
+    # oracle: output rows [0, 1024) of the decode problem per call
+    ORACLE_ROWS = 1024
+
+    def oracle_setup(self):
+        import oracle as oracle_pkg
+        from bit_linear_layers_b200 import synthetic
+        self.o = oracle_pkg.get()
+        W = synthetic.weights(self.N, self.K, seed=2).numpy()
+        self.ox = synthetic.bf16_bits(synthetic.activations(self.M, self.K, seed=2))
+        packed, alpha = self.o.pack_fbi(W)
+        self.op, self.oa = packed[:self.ORACLE_ROWS].copy(), alpha[:self.ORACLE_ROWS].copy()
+        self.oracle_sample = (f"output rows 0..{self.ORACLE_ROWS - 1} of the 1x4096x4096 problem per call "
+                              "(single-threaded C oracle, fp64)")
+        return self.ORACLE_ROWS * self.K / 8  # units (packed bytes) per call
+
+    def oracle_call(self):
+        self.o.w1a16(self.ox, self.op, self.oa, self.K)
+
+
+class Prefill(Workload):
+    name = "prefill"
+    SHAPES = [(2048, 4096, 11008), (2048, 11008, 4096)]  # (M, K, N)
+    metric = "prefill TFLOP/s (W1A16, 7B MLP up + down projections, 2048 tokens)"
+    unit, scale, bound = "TFLOP/s", 1e12, "tensor"
+    kernel = "gemm_ts_kernel<0,1,256,false> (persistent, 148 CTAs)"
+    sources = [CSRC + "bl_gemm_ts.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = "gemm_ts_w1a16_prefill_2048x4096x11008.traffic.json"
+    launches_per_step = 2
+    rotate = 4
+
+    def __init__(self):
+        per_copy = sum(M * K * 2 + N * K // 8 + 4 * N + M * N * 2 for M, K, N in self.SHAPES)
+        self.config = {"workload": "FBI-linear W1A16 prefill GEMM, 2048 tokens, 7B MLP shapes "
+                                   "4096->11008 then 11008->4096",
+                       "shapes_MKN": [list(s) for s in self.SHAPES],
+                       "l2": f"inputs larger than L2: {self.rotate} distinct copies of weights, activations "
+                             f"and outputs ({self.rotate * per_copy / 1e6:.0f} MB) rotated step to step"}
+
+    def units_per_step(self):
+        return sum(2.0 * M * K * N for M, K, N in self.SHAPES)
+
+    def peak(self, peaks, timed_s):
+        key = "bf16_tflops_sustained" if timed_s > SUSTAINED_AFTER_S else "bf16_tflops"
+        return peaks[key], key
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        from bit_linear_layers_b200 import synthetic
+        self.bl = bl
+        self.copies = []
+        for i in range(self.rotate):
+            layers = []
+            for s, (M, K, N) in enumerate(self.SHAPES):
+                seed = 1 + 100 * i + 10 * s + 7 * rank
+                W = synthetic.weights(N, K, seed=seed, device=dev)
+                p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
+                del W
+                x = synthetic.activations(M, K, seed=seed, device=dev)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                layers.append((x, p, a, y))
+            self.copies.append(layers)
+        self.xh = [lay[0].cpu().pin_memory() for lay in self.copies[0]]
+        self.yh = [torch.empty_like(lay[3], device="cpu").pin_memory() for lay in self.copies[0]]
+        self.h2d = sum(M * K * 2 for M, K, N in self.SHAPES)
+        self.d2h = sum(M * N * 2 for M, K, N in self.SHAPES)
+
+    def step(self, i):
+        for x, p, a, y in self.copies[i % self.rotate]:
+            self.bl.bin_linear_w1a16(x, p, a, out=y)
+
+    def e2e_step(self, i):
+        for (x, p, a, y), xh, yh in zip(self.copies[i % self.rotate], self.xh, self.yh):
+            x.copy_(xh, non_blocking=True)
+            self.bl.bin_linear_w1a16(x, p, a, out=y)
+            yh.copy_(y, non_blocking=True)
+
+    # oracle: one token through output columns [0, 512) of the up and [0, 256) of the down projection
+    ORACLE_COLS = (512, 256)
+
+    def oracle_setup(self):
+        import oracle as oracle_pkg
+        from bit_linear_layers_b200 import synthetic
+        self.o = oracle_pkg.get()
+        self.olayers, flop = [], 0.0
+        for s, ((M, K, N), cols) in enumerate(zip(self.SHAPES, self.ORACLE_COLS)):
+            W = synthetic.weights(cols, K, seed=1 + 10 * s).numpy()  # `cols` rows of a seeded layer
+            x = synthetic.bf16_bits(synthetic.activations(1, K, seed=1 + 10 * s))
+            p, a = self.o.pack_fbi(W)
+            self.olayers.append((x, p, a, K))
+            flop += 2.0 * K * cols
+        self.oracle_sample = ("one token through output columns 0..511 of the up and 0..255 of the down "
+                              "projection per call (single-threaded C oracle, fp64)")
+        return flop
+
+    def oracle_call(self):
+        for x, p, a, K in self.olayers:
+            self.o.w1a16(x, p, a, K)
+
+
+class W1A8(Workload):
+    name = "w1a8"
+    SHAPES = [(512, 2048, 5632), (512, 5632, 2048)]
+    metric = "BitLinear W1A8 TOP/s (1.3B shapes, 512 tokens, LN + absmax quant + int8 GEMM + rescale)"
+    unit, scale, bound = "TOP/s", 1e12, "tensor"
+    dtype = "s8"
+    kernel = "ln_quant_kernel + gemm_ts_kernel<1,2,128,*> (one call; time includes LN + quantisation)"
+    sources = [CSRC + "bl_gemm_ts.cuh", CSRC + "bl_lnquant.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = None
+    launches_per_step = 4
+    rotate = 16
+
+    def __init__(self):
+        per_copy = sum(M * K * 2 + N * K // 8 + M * K + 8 * M + M * N * 4 for M, K, N in self.SHAPES)
+        self.config = {"workload": "BitNet BitLinear W1A8, 512 tokens, 1.3B shapes 2048->5632 then 5632->2048",
+                       "shapes_MKN": [list(s) for s in self.SHAPES],
+                       "l2": f"inputs larger than L2: {self.rotate} distinct copies of weights, activations, "
+                             f"workspaces and outputs ({self.rotate * per_copy / 1e6:.0f} MB) rotated step to step"}
+
+    def units_per_step(self):
+        return sum(2.0 * M * K * N for M, K, N in self.SHAPES)
+
+    def peak(self, peaks, timed_s):
+        key = "bf16_tflops_sustained" if timed_s > SUSTAINED_AFTER_S else "bf16_tflops"
+        return 2.0 * peaks[key], f"2 x {key} (nominal int8/bf16 ratio)"
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        from bit_linear_layers_b200 import synthetic
+        self.bl = bl
+        self.copies = []
+        for i in range(self.rotate):
+            layers = []
+            for s, (M, K, N) in enumerate(self.SHAPES):
+                seed = 4 + 100 * i + 10 * s + 7 * rank
+                W = synthetic.weights(N, K, seed=seed, mean=0.001, device=dev)
+                p, _, b = bl.bin_pack(W, bl.BL_PACK_BITNET)
+                del W
+                x = synthetic.laplace_channel_activations(M, K, seed=seed, device=dev)
+                ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W1A8, M, N, K), dtype=torch.uint8, device=dev)
+                y = torch.empty((M, N), dtype=torch.float32, device=dev)
+                layers.append((x, p, b, ws, y))
+            self.copies.append(layers)
+        self.xh = [lay[0].cpu().pin_memory() for lay in self.copies[0]]
+        self.yh = [torch.empty_like(lay[4], device="cpu").pin_memory() for lay in self.copies[0]]
+        self.h2d = sum(M * K * 2 for M, K, N in self.SHAPES)
+        self.d2h = sum(M * N * 4 for M, K, N in self.SHAPES)
+
+    def step(self, i):
+        for x, p, b, ws, y in self.copies[i % self.rotate]:
+            self.bl.bitlinear_w1a8(x, p, b, out=y, ws=ws)
+
+    def e2e_step(self, i):
+        for (x, p, b, ws, y), xh, yh in zip(self.copies[i % self.rotate], self.xh, self.yh):
+            x.copy_(xh, non_blocking=True)
+            self.bl.bitlinear_w1a8(x, p, b, out=y, ws=ws)
+            yh.copy_(y, non_blocking=True)
+
+    # oracle: token 0 through output columns [0, 1024) of both projections
+    ORACLE_COLS = 1024
+
+    def oracle_setup(self):
+        import oracle as oracle_pkg
+        from bit_linear_layers_b200 import synthetic
+        self.o = oracle_pkg.get()
+        self.olayers, ops = [], 0.0
+        for s, (M, K, N) in enumerate(self.SHAPES):
+            W = synthetic.weights(N, K, seed=4 + 10 * s, mean=0.001).numpy()
+            p, _, beta = self.o.pack_bitnet(W)  # beta needs the whole matrix
+            x = synthetic.bf16_bits(synthetic.laplace_channel_activations(1, K, seed=4 + 10 * s))
+            self.olayers.append((x, p[:self.ORACLE_COLS].copy(), beta, K))
+            ops += 2.0 * K * self.ORACLE_COLS
+        self.oracle_sample = ("one token through LN + quantisation and output columns 0..1023 of both "
+                              "projections per call (single-threaded C oracle, fp64/int64)")
+        return ops
+
+    def oracle_call(self):
+        for x, p, beta, K in self.olayers:
+            self.o.w1a8(x, p, beta, K)
+
+
+WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8)}
+
+
 # ----------------------------------------------------------------------------- ours
 
 
-def run_ours(args, rank, world, local_rank):
+def _capture(step, first, count, stream):
     import torch
-    import bit_linear_layers_b200 as bl
-    from bit_linear_layers_b200 import synthetic
-
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    M, K, N = M_DEC, K_DEC, N_DEC
-    # weights: copy 0 is the seeded workload (CPU generator), the others are
-    # further seeded draws made on the device
-    packs, alphas, xs = [], [], []
-    for i in range(ROTATE):
-        if i == 0:
-            W = synthetic.weights(N, K, seed=2).to(dev)
-            x = synthetic.activations(M, K, seed=2).to(dev)
-        else:
-            W = synthetic.weights(N, K, seed=2 + 1000 * i + 7 * rank, device=dev)
-            x = synthetic.activations(M, K, seed=2 + 1000 * i + 7 * rank, device=dev)
-        p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
-        packs.append(p)
-        alphas.append(a)
-        xs.append(x)
-        del W
-    ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(ROTATE)]
-    torch.cuda.synchronize()
-
-    # consecutive steps never write each other's weights, so each launch may
-    # start streaming its weights while the previous one finishes
-    flags = bl.BL_FLAG_OVERLAP_PREVIOUS
-
-    def step(i):
-        j = i % ROTATE
-        bl.bin_linear_w1a16(xs[j], packs[j], alphas[j], out=ys[j], flags=flags)
-
-    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
-    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else local_rank)
-    sampler.start()
-    # settle clocks (untimed), then exactly W warm-up steps
-    t_end = time.time() + 1.0
-    while time.time() < t_end:
-        for i in range(256):
-            step(i)
-        torch.cuda.synchronize()
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-
-    K_steps = args.steps
     graph = torch.cuda.CUDAGraph()
-    stream = torch.cuda.Stream(device=dev)
-    stream.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(stream):
         with torch.cuda.graph(graph, stream=stream):
-            for i in range(K_steps):
-                step(args.warmup + i)
+            for i in range(count):
+                step(first + i)
     torch.cuda.synchronize()
     graph.replay()  # untimed replay: the graph's first launch uploads it
     torch.cuda.synchronize()
+    return graph
 
+
+def _timed_replay(graph, dev, world):
+    import torch
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -207,143 +456,77 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    ms = e0.elapsed_time(e1)
+    return e0.elapsed_time(e1)
 
-    # end to end through host buffers: x from pinned host, y back to pinned host
-    xh = [x.cpu().pin_memory() for x in xs]
-    yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(ROTATE)]
-    xd = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    yd = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
 
-    def e2e_step(i):
-        j = i % ROTATE
-        xd.copy_(xh[j], non_blocking=True)
-        bl.bin_linear_w1a16(xd, packs[j], alphas[j], out=yd, flags=flags)
-        yh[j].copy_(yd, non_blocking=True)
+def run_workload(wl, steps, warmup, rank, world, dev, sampler=None):
+    """Device-resident and end-to-end times (ms) of `steps` steps, max over ranks."""
+    import torch
+    wl.setup(dev, rank)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.start()
+    # settle clocks (untimed, about a second), then exactly W warm-up steps
+    t_end, i = time.time() + 1.0, 0
+    while time.time() < t_end:
+        for _ in range(max(1, 256 // wl.launches_per_step)):
+            wl.step(i)
+            i += 1
+        torch.cuda.synchronize()
+    for i in range(warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
 
-    for i in range(args.warmup):
-        e2e_step(i)
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    graph = _capture(wl.step, warmup, steps, stream)
+    ms = _timed_replay(graph, dev, world)
+    del graph
+
+    for i in range(warmup):
+        wl.e2e_step(i)
     torch.cuda.synchronize()
-    g2 = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(g2, stream=stream):
-            for i in range(K_steps):
-                e2e_step(i)
-    g2.replay()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0.record(launch_stream)
-    g2.replay()
-    e1.record(launch_stream)
-    torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    clocks = sampler.stop()
+    g2 = _capture(wl.e2e_step, warmup, steps, stream)
+    ms_e2e = _timed_replay(g2, dev, world)
+    del g2
+    clocks = sampler.stop() if sampler is not None else None
 
     if world > 1:
         t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms, ms_e2e = float(t[0]), float(t[1])
-    del graph, g2
     return ms, ms_e2e, clocks
 
 
-def cpu_baseline_decode(target_s=10.0, cap_s=30.0):
-    import numpy as np
-    import oracle as oracle_pkg
-    from bit_linear_layers_b200 import synthetic
-
-    o = oracle_pkg.get()
-    W = synthetic.weights(N_DEC, K_DEC, seed=2).numpy()
-    x = synthetic.bf16_bits(synthetic.activations(M_DEC, K_DEC, seed=2))
-    packed, alpha = o.pack_fbi(W)
+def cpu_baseline(wl, target_s=10.0):
+    """The oracle as it stands, on the host, over repeated bounded samples."""
+    units = wl.oracle_setup()
     reps, t0 = 0, time.perf_counter()
     while True:
-        o.w1a16(x, packed, alpha, K_DEC)
+        wl.oracle_call()
         reps += 1
         el = time.perf_counter() - t0
-        if el >= target_s or el >= cap_s:
+        if el >= target_s:
             break
-    gbs = reps * (N_DEC * K_DEC / 8) / el / 1e9
-    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"the full 1x4096x4096 decode problem, {reps} calls in {el:.1f} s "
-                      "(single-threaded C oracle, fp64)"}, np
+    return {"value": reps * units / el / wl.scale, "unit": wl.unit, "cores": 1, "kind": "oracle",
+            "sample": f"{wl.oracle_sample}; {reps} calls in {el:.1f} s"}
 
 
-# ----------------------------------------------------------------------------- secondary
-
-def _flush_buffer(dev):
-    import torch
-    return torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MB > 126 MB L2
-
-
-def _timed_call(fn, flush, reps=5):
-    """Median device time (ms) of fn() with L2 flushed before every call."""
-    import torch
-    ts = []
-    for _ in range(2):
-        fn()
-    for _ in range(reps):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        fn()
-        e1.record()
-        torch.cuda.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    ts.sort()
-    return ts[len(ts) // 2]
-
-
-def secondary_prefill(dev, peaks, flush):
-    """W1A16 prefill on the 7B MLP shapes: TFLOPS vs the measured bf16 peak."""
-    import bit_linear_layers_b200 as bl
-    from bit_linear_layers_b200 import synthetic
-    out, total_flop, total_ms = [], 0.0, 0.0
-    for (M, K, N) in [(2048, 4096, 11008), (2048, 11008, 4096)]:
-        W = synthetic.weights(N, K, seed=1, device=dev)
-        x = synthetic.activations(M, K, seed=1, device=dev)
-        p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
-        del W
-        ms = _timed_call(lambda: bl.bin_linear_w1a16(x, p, a), flush)
-        flop = 2.0 * M * N * K
-        out.append({"shape": f"{M}x{K}x{N}", "us": ms * 1e3, "tflops": flop / (ms * 1e-3) / 1e12})
-        total_flop += flop
-        total_ms += ms
-    tf = total_flop / (total_ms * 1e-3) / 1e12
-    return {"metric": "prefill TFLOPS (W1A16, 7B MLP shapes, 2048 tokens)", "tflops": tf,
-            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": tf / peaks["bf16_tflops"], "kernel": "gemm_ts_kernel<0,128>",
-                         "peak_source": "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops)"},
-            "shapes": out, "l2": "flushed (256 MB write) before every call"}
-
-
-def secondary_w1a8(dev, peaks, flush):
-    """BitLinear W1A8 at the 1.3B shapes (512 tokens): LN+quant and int8 GEMM."""
-    import torch
-    import bit_linear_layers_b200 as bl
-    from bit_linear_layers_b200 import synthetic
-    int8_peak = 2.0 * peaks["bf16_tflops"]
-    out, total_op, total_ms = [], 0.0, 0.0
-    for (M, K, N) in [(512, 2048, 5632), (512, 5632, 2048)]:
-        W = synthetic.weights(N, K, seed=4, mean=0.001, device=dev)
-        x = synthetic.laplace_channel_activations(M, K, seed=4, device=dev)
-        p, _, b = bl.bin_pack(W, bl.BL_PACK_BITNET)
-        del W
-        ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W1A8, M, N, K), dtype=torch.uint8, device=dev)
-        y = torch.empty((M, N), dtype=torch.float32, device=dev)
-        ms = _timed_call(lambda: bl.bitlinear_w1a8(x, p, b, out=y, ws=ws), flush)
-        op = 2.0 * M * N * K
-        out.append({"shape": f"{M}x{K}x{N}", "us": ms * 1e3, "tops": op / (ms * 1e-3) / 1e12})
-        total_op += op
-        total_ms += ms
-    tops = total_op / (total_ms * 1e-3) / 1e12
-    return {"metric": "BitLinear W1A8 TOPS (1.3B shapes, 512 tokens, LN + quant + int8 GEMM)", "tops": tops,
-            "roofline": {"bound": "tensor", "achieved": tops, "peak": int8_peak, "unit": "TOP/s",
-                         "frac": tops / int8_peak,
-                         "peak_source": "measured bf16 burst x nominal int8/bf16 ratio 2"},
-            "shapes": out, "l2": "flushed (256 MB write) before every call"}
+def summarize(wl, ms, ms_e2e, steps, world, peaks, peak_kind):
+    per_step_s = ms * 1e-3 / steps
+    timed_s = ms * 1e-3
+    peak, peak_key = wl.peak(peaks, timed_s)
+    achieved = wl.achieved(per_step_s)
+    roof = {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": wl.unit,
+            "frac": achieved / peak, "traffic": wl.traffic(), "kernel": wl.kernel,
+            "peak_source": f"{peak_kind}: MEASURED_PEAKS.json {peak_key}" if peak_kind == "measured"
+            else f"fallback ({peak_key})"}
+    if isinstance(wl, Decode):
+        roof["algorithmic_bytes_per_launch"] = wl.alg_b
+    value = world * steps * wl.units_per_step() / timed_s / wl.scale
+    e2e = {"value": world * steps * wl.units_per_step() / (ms_e2e * 1e-3) / wl.scale, "unit": wl.unit,
+           "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h, "ms_per_step": ms_e2e / steps}
+    return value, roof, e2e
 
 
 def secondary_llama7b(dev, peaks):
@@ -367,7 +550,6 @@ def secondary_llama7b(dev, peaks):
     res = {"packed_GB": packed_bytes / 1e9}
     for B in (1, 16):
         x = synthetic.activations(B, 4096, seed=77, device=dev)
-        bufs = {n: torch.empty((B, n), dtype=torch.bfloat16, device=dev) for n in (4096, 11008)}
         q, k, v, o = (torch.empty((B, 4096), dtype=torch.bfloat16, device=dev) for _ in range(4))
         g, u = (torch.empty((B, 11008), dtype=torch.bfloat16, device=dev) for _ in range(2))
         h = torch.empty((B, 4096), dtype=torch.bfloat16, device=dev)
@@ -438,10 +620,108 @@ def secondary_llama7b(dev, peaks):
     return res
 
 
-def bytes_per_step():
-    packed = N_DEC * K_DEC // 8
-    alg = packed + 4 * N_DEC + 2 * M_DEC * K_DEC + 2 * M_DEC * N_DEC
-    return packed, alg
+def secondary(args, dev, peaks, peak_kind):
+    """The workloads other than the headline one, 200 steps each, plus the
+    7B-shaped model. Only at N=1."""
+    import gc
+    import torch
+    out = {}
+    for name, cls in WORKLOADS.items():
+        if name == args.workload:
+            continue
+        wl = cls()
+        steps = 200
+        ms, ms_e2e, _ = run_workload(wl, steps, 3, 0, 1, dev)
+        value, roof, e2e = summarize(wl, ms, ms_e2e, steps, 1, peaks, peak_kind)
+        out[name] = {"metric": wl.metric, "value": value, "unit": wl.unit, "ms_per_step": ms / steps,
+                     "steps": steps, "warmup": 3, "config": wl.config, "roofline": roof, "e2e": e2e,
+                     "gpu_launches": steps * wl.launches_per_step}
+        del wl
+        gc.collect()
+        torch.cuda.empty_cache()
+    out["pack"] = secondary_pack(dev, peaks)
+    out["decode_l2_warm"] = secondary_decode_warm(dev)
+    out["llama7b_linear"] = secondary_llama7b(dev, peaks)
+    return out
+
+
+def secondary_pack(dev, peaks):
+    """bin_pack of a 4096 x 11008 fp32 matrix (180 MB, more than L2) in both
+    modes: GB/s on the bytes it must move (W read, packed bits and scales written)."""
+    import torch
+    import bit_linear_layers_b200 as bl
+    from bit_linear_layers_b200 import synthetic
+    N, K = 11008, 4096
+    W = synthetic.weights(N, K, seed=6, device=dev)
+    res = {}
+    for mode, name in ((bl.BL_PACK_FBI, "fbi"), (bl.BL_PACK_BITNET, "bitnet")):
+        packed = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
+        alpha = torch.empty(N if mode == bl.BL_PACK_FBI else 1, dtype=torch.float32, device=dev)
+        beta = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(max(1, bl.workspace_bytes(bl.BL_OP_PACK_BITNET if mode else bl.BL_OP_PACK_FBI, 0, N, K)),
+                         dtype=torch.uint8, device=dev)
+
+        def call():
+            bl.bin_pack(W, mode, packed=packed, alpha=alpha, beta=beta, ws=ws)
+
+        ms = _median_ms(call, reps=10)
+        nbytes = 4 * N * K + N * K // 8 + 4 * alpha.numel()
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"shape_NK": [N, K], "us": ms * 1e3, "GB_s": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                     "launches": 1 if mode == bl.BL_PACK_FBI else 3}
+    res["l2"] = "W is 180 MB, more than L2"
+    return res
+
+
+def secondary_decode_warm(dev):
+    """Single-launch latency of the decode GEMV with no rotation (weights
+    L2-warm), one launch per step in a CUDA graph, with and without
+    programmatic dependent launch."""
+    import torch
+    import bit_linear_layers_b200 as bl
+    from bit_linear_layers_b200 import synthetic
+    W = synthetic.weights(4096, 4096, seed=2, device=dev)
+    p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
+    x = synthetic.activations(1, 4096, seed=2, device=dev)
+    y = torch.empty((1, 4096), dtype=torch.bfloat16, device=dev)
+    res = {"label": "L2-warm: the same 2 MB of weights every launch"}
+    for flags, name in ((0, "plain"), (bl.BL_FLAG_OVERLAP_PREVIOUS, "overlap_previous")):
+        reps = 200
+        st = torch.cuda.Stream(device=dev)
+        st.wait_stream(torch.cuda.current_stream(dev))
+        for _ in range(5):
+            bl.bin_linear_w1a16(x, p, a, out=y, flags=flags)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(g, stream=st):
+                for _ in range(reps):
+                    bl.bin_linear_w1a16(x, p, a, out=y, flags=flags)
+        g.replay()
+        torch.cuda.synchronize()
+        res[f"{name}_us_per_launch"] = _median_ms(g.replay, reps=5) * 1e3 / reps
+        del g
+    return res
+
+
+def _median_ms(fn, reps=5):
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    return ts[len(ts) // 2]
+
+
+# ----------------------------------------------------------------------------- main
 
 
 def main():
@@ -449,39 +729,29 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    packed_b, alg_b = bytes_per_step()
-    metric = "decode GEMV HBM GB/s on packed-weight bytes (W1A16, 1x4096x4096)"
-    config = {"workload": "FBI-linear W1A16 decode GEMV, M=1, K=4096, N=4096 (7B attention projection)",
-              "M": M_DEC, "K": K_DEC, "N": N_DEC,
-              "l2": f"inputs larger than L2: {ROTATE} distinct packed weight copies "
-                    f"({ROTATE * packed_b / 1e6:.0f} MB) rotated step to step",
-              "timing": "K steps in one CUDA graph, CUDA events on the launching stream",
-              "launch": "programmatic dependent launch between steps (BL_FLAG_OVERLAP_PREVIOUS)",
-              "parallelism": f"replicas x{world}"}
+    wl = WORKLOADS[args.workload]()
+    config = dict(wl.config)
+    config["timing"] = "K steps in one CUDA graph, CUDA events on the launching stream"
+    config["parallelism"] = f"replicas x{world}"
 
     if args.impl == "reference":
         if rank != 0:
             return 0
-        import oracle as oracle_pkg
-        from bit_linear_layers_b200 import synthetic
-        o = oracle_pkg.get()
-        W = synthetic.weights(N_DEC, K_DEC, seed=2).numpy()
-        x = synthetic.bf16_bits(synthetic.activations(M_DEC, K_DEC, seed=2))
-        packed, alpha = o.pack_fbi(W)
+        units = wl.oracle_setup()
         for _ in range(args.warmup):
-            o.w1a16(x, packed, alpha, K_DEC)
+            wl.oracle_call()
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            o.w1a16(x, packed, alpha, K_DEC)
+            wl.oracle_call()
         el = time.perf_counter() - t0
-        value = args.steps * packed_b / el / 1e9
-        line = {"impl": "reference", "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world,
+        value = args.steps * units / el / wl.scale
+        line = {"impl": "reference", "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": config,
-                "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                 "sample": f"the full decode problem once per step, {args.steps} steps"},
-                "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+                "cpu_baseline": {"value": value, "unit": wl.unit, "cores": 1, "kind": "oracle",
+                                 "sample": f"{wl.oracle_sample}; one call per step"},
+                "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
 
@@ -490,41 +760,30 @@ def main():
         import datetime
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    ms, ms_e2e, clocks = run_ours(args, rank, world, local_rank)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else local_rank)
+    ms, ms_e2e, clocks = run_workload(wl, args.steps, args.warmup, rank, world, dev, sampler)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
         return 0
     peaks, peak_kind = load_peaks()
-    per_step_ms = ms / args.steps
-    value = world * args.steps * packed_b / (ms * 1e-3) / 1e9
-    achieved = alg_b / (per_step_ms * 1e-3) / 1e9
-    cpu, _ = cpu_baseline_decode()
-    secondary = None
+    value, roof, e2e = summarize(wl, ms, ms_e2e, args.steps, world, peaks, peak_kind)
+    cpu = cpu_baseline(wl) if world == 1 else None
+    extra = None
     if world == 1 and not args.no_secondary:
-        import torch
-        dev = torch.device("cuda", local_rank)
-        flush = _flush_buffer(dev)
-        secondary = {"prefill_w1a16": secondary_prefill(dev, peaks, flush),
-                     "w1a8_1p3b": secondary_w1a8(dev, peaks, flush)}
-        del flush
-        secondary["llama7b_linear"] = secondary_llama7b(dev, peaks)
+        del wl
+        torch.cuda.empty_cache()
+        extra = secondary(args, dev, peaks, peak_kind)
     line = {
-        "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_per_launch(),
-                     "kernel": "gemv_w1a16_lut_kernel<1> (cluster of 8 x 16 clusters)", "algorithmic_bytes_per_launch": alg_b,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                     else "fallback 6.65 TB/s"},
-        "cpu_baseline": cpu,
-        "e2e": {"value": world * args.steps * packed_b / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
-                "h2d_bytes_per_step": 2 * M_DEC * K_DEC, "d2h_bytes_per_step": 2 * M_DEC * N_DEC,
-                "ms_per_step": ms_e2e / args.steps},
-        "gpu_launches": args.steps,
-        "clocks": clocks,
-        "secondary": secondary,
+        "metric": WORKLOADS[args.workload].metric, "value": value, "unit": roof["unit"], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": WORKLOADS[args.workload].dtype, "data": "synthetic",
+        "config": config, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps * WORKLOADS[args.workload].launches_per_step,
+        "clocks": clocks, "secondary": extra,
     }
     print(json.dumps(line), flush=True)
     return 0

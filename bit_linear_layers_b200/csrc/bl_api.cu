@@ -192,11 +192,11 @@ int launch_ts_cfg(const CUtensorMap& tm_x, const CUtensorMap& tm_bits, int64_t M
     }
     return launch_status();
   }
-  // persistent: output tile written by one bulk tensor store when the row pitch allows it
+  // persistent: output tile written by bulk tensor stores when the row pitch allows it
   const int use_tma_store =
-      (N * C::OUT_ELEM) % 16 == 0 &&
+      C::STAGE_OUT && (N * C::OUT_ELEM) % 16 == 0 &&
       make_map_2d(&tm_y, y, KIND == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                  C::OUT_ELEM, uint64_t(N), uint64_t(M), C::ROWS, T, CU_TENSOR_MAP_SWIZZLE_NONE);
+                  C::OUT_ELEM, uint64_t(N), uint64_t(M), C::STAGE_COLS, T, CU_TENSOR_MAP_SWIZZLE_NONE);
   const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
   gemm_ts_kernel<KIND, NB, T, SPLIT><<<grid, kTsThreads, C::SMEM_BYTES, s>>>(
       tm_x, tm_bits, tm_y, use_tma_store, int(M), int(N), int(K), alpha, gamma, beta, y, acc_out);

@@ -5,7 +5,7 @@
 //     y[m][j] = bf16( alpha_j * sum_k s_jk x[m][k] )          kind::f16, fp32 accumulate
 //   W1A8 ("BitNet b1.58" page, section 1, Eq.(7)-(8)):
 //     acc[m][j] = sum_k s_jk q[m][k]  (exact int32)            kind::i8
-//     y[m][j]   = fp32( acc * beta * gamma_m / 128 )           fp64 epilogue
+//     y[m][j]   = fp32( acc * beta * gamma_m / 128 )           per-token scale in fp64
 //
 // The product is computed transposed, D[j][m] = sum_k S[j][k] X[m][k]: the
 // 1-bit weights are the MMA's M side (NB blocks of 128 rows per tile), the
@@ -61,10 +61,16 @@ struct TsCfg {
   static constexpr int BITS_BYTES = ROWS * 16;                  // one 128-k sign stage
   static constexpr int SB = 4;                                  // sign stages in shared memory
   static constexpr int OUT_ELEM = KIND == 0 ? 2 : 4;            // y element bytes
-  // the output tile is staged for one bulk store when it fits in 64 KB
-  static constexpr bool STAGE_OUT = !SPLIT && ROWS * T * OUT_ELEM <= 64 * 1024;
-  // staged output tile [T][ROWS], or the split-K inbox of 4-byte partials [S][ROWS/S][T]
-  static constexpr int OUT_BYTES = SPLIT ? ROWS * T * 4 : (STAGE_OUT ? ROWS * T * OUT_ELEM : 0);
+  // the output tile is staged in shared memory and written by bulk tensor
+  // stores: the whole tile at once when it fits in 64 KB, else one 128-row
+  // block at a time
+  static constexpr int STAGE_COLS = ROWS * T * OUT_ELEM <= 64 * 1024 ? ROWS : 128;
+  static constexpr bool STAGE_OUT = !SPLIT && STAGE_COLS * T * OUT_ELEM <= 64 * 1024;
+  // split-K inbox rows: T partials padded by 16 bytes, so that a warp's
+  // 16-byte reads of consecutive rows spread over all banks
+  static constexpr int IN_STRIDE = T + 4;
+  // staged output [T][STAGE_COLS], or the split-K inbox [S][ROWS/S][IN_STRIDE] of 4-byte partials
+  static constexpr int OUT_BYTES = SPLIT ? ROWS * IN_STRIDE * 4 : (STAGE_OUT ? STAGE_COLS * T * OUT_ELEM : 0);
   static constexpr int SX_FIT = (210 * 1024 - OUT_BYTES - SB * BITS_BYTES) / X_UNIT_BYTES;
   static constexpr int SX = SX_FIT > 8 ? 8 : SX_FIT;           // activation units in flight
   static constexpr int X_RING = SX * X_UNIT_BYTES;
@@ -119,6 +125,17 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // barrier among the four epilogue warps only
 __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// the same barrier, returning the AND of every epilogue thread's `v`
+__device__ __forceinline__ bool epilogue_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
 
 // D(tmem) (+)= A(tmem) * B(smem desc)
 __device__ __forceinline__ void umma_ts_bf16(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -154,6 +171,38 @@ __device__ __forceinline__ void expand16_i8(uint32_t bits, uint32_t* out) {
   }
 }
 
+// W1A8 output y = acc * s, s = beta * gamma_m / 128 formed in fp64 once per
+// token and carried as two floats (s = hi + lo to about 2^-48). For
+// |acc| < 2^22 the product is evaluated in fp32 with an error-free product
+// (the magic-number add turns acc into a float exactly, the fma recovers the
+// rounding error of acc * hi), so y is the fp32 rounding of the exact value
+// except within ~2^-46 of a rounding midpoint; larger |acc| take fp64.
+struct TokScale {
+  float hi, lo;
+};
+__device__ __forceinline__ TokScale w1a8_token_scale(double beta, double gamma) {
+  const double sc = beta * gamma * 0.0078125;  // division by 128 = exact scaling by 2^-7
+  const float hi = static_cast<float>(sc);
+  return TokScale{hi, static_cast<float>(sc - static_cast<double>(hi))};
+}
+constexpr int32_t kW1a8FastLimit = 1 << 22;
+__device__ __forceinline__ bool w1a8_fast_ok(int32_t acc) {
+  return acc > -kW1a8FastLimit && acc < kW1a8FastLimit;
+}
+// |acc| < 2^22 only (no branch, so that unrolled loops interleave)
+__device__ __forceinline__ float w1a8_output_fast(int32_t acc, TokScale s) {
+  const float a = __int_as_float(0x4B400000 + acc) - 12582912.0f;  // exact: 1.5 * 2^23 + acc - 1.5 * 2^23
+  const float p = a * s.hi;
+  const float e = fmaf(a, s.hi, -p);  // a * hi - p, exactly
+  return p + fmaf(a, s.lo, e);
+}
+__device__ __forceinline__ float w1a8_output_wide(int32_t acc, TokScale s) {
+  return static_cast<float>(static_cast<double>(acc) * (static_cast<double>(s.hi) + static_cast<double>(s.lo)));
+}
+__device__ __forceinline__ float w1a8_output(int32_t acc, TokScale s) {
+  return w1a8_fast_ok(acc) ? w1a8_output_fast(acc, s) : w1a8_output_wide(acc, s);
+}
+
 __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, const uint32_t* v, uint32_t remote_bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
                    remote_addr),
@@ -187,6 +236,10 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
   __shared__ __align__(8) uint64_t a_full[SA], a_empty[SA], d_full, d_empty;
   __shared__ uint32_t tmem_base_sh;
   __shared__ __align__(8) uint64_t inbox_bar;
+  // epilogue scales staged once per tile: beta * gamma / 128 of the tile's tokens (W1A8),
+  // alpha of the rows a split-K owner finishes (W1A16)
+  __shared__ TokScale tok_scale[KIND == 1 ? T : 1];
+  __shared__ float row_alpha[SPLIT && KIND == 0 ? ROWS : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_kb = K / kTsStageK;
@@ -369,22 +422,34 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     }
   } else if (warp >= 4 && SPLIT) {
     // ---------------- split-K epilogue: push partials, owner reduces ----------------
-    const int q = warp & 3;
+    const int q = warp & 3, et = threadIdx.x - 128;
     const int rows_per = ROWS / S;                      // rows owned by each CTA of the cluster
-    uint8_t* inbox = bits_ring + C::SB * C::BITS_BYTES;  // [S][rows_per][T] 4-byte partials
+    constexpr int IN_STRIDE = C::IN_STRIDE;             // 4-byte words per inbox row
+    uint8_t* inbox = bits_ring + C::SB * C::BITS_BYTES;  // [S][rows_per][IN_STRIDE] 4-byte partials
     const int tile = tile_first;
     const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
-    bool ok = true;
+    // scales of the rows this CTA finishes / of the tile's tokens, read while the MMAs run
+    if (KIND == 1) {
+      const double bt = static_cast<double>(*beta);
+      for (int tt = et; tt < T; tt += 128)
+        tok_scale[tt] = w1a8_token_scale(bt, t0 + tt < M ? gamma[t0 + tt] : 0.0);
+    } else {
+      for (int rr = et; rr < rows_per; rr += 128) {
+        const int j = w0 + static_cast<int>(rank) * rows_per + rr;
+        row_alpha[rr] = j < N ? alpha[j] : 0.f;
+      }
+    }
     if (threadIdx.x == 128) mbar_arrive_expect_tx(smem_u32(&inbox_bar), ROWS * T * 4);
     asm volatile("barrier.cluster.wait;" ::: "memory");  // every inbox barrier is initialised
-    if (!mbar_wait(smem_u32(&d_full), 0, kWhereGemmEpilogue)) ok = false;
+    // warp-uniform outcome: the TMEM loads below are warp-collective
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&d_full), 0, kWhereGemmEpilogue));
     tc_fence_after_sync();
 #pragma unroll 1
     for (int blk = 0; blk < NB && ok; ++blk) {
       const int jl = blk * 128 + q * 32 + lane;
       const uint32_t owner = static_cast<uint32_t>(jl / rows_per);
       const uint32_t slot0 =
-          smem_u32(inbox + (static_cast<int>(rank) * rows_per + jl % rows_per) * T * 4);
+          smem_u32(inbox + (static_cast<int>(rank) * rows_per + jl % rows_per) * IN_STRIDE * 4);
       const uint32_t rslot = ts_map_rank(slot0, owner);
       const uint32_t rbar = ts_map_rank(smem_u32(&inbox_bar), owner);
 #pragma unroll 1
@@ -397,104 +462,150 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
         for (int v = 0; v < 8; ++v) st_async_v4(rslot + (cc * 32 + v * 4) * 4, r + v * 4, rbar);
       }
     }
-    // owner: add the S partials of its rows in rank order, then scale and store
-    if (ok && mbar_wait(smem_u32(&inbox_bar), 0, kWhereGemmEpilogue)) {
-      const int et = threadIdx.x - 128;  // 0..127
-      double bt = 0.0;
-      if (KIND == 1) bt = static_cast<double>(*beta);
-      for (int e = et; e < rows_per * T; e += 128) {
-        const int rr = e % rows_per, tt = e / rows_per;
-        const int j = w0 + static_cast<int>(rank) * rows_per + rr, m = t0 + tt;
-        if (j >= N || m >= M) continue;
-        const int64_t o = static_cast<int64_t>(m) * N + j;
-        if (KIND == 0) {
-          float acc = 0.f;
-          for (int src = 0; src < S; ++src)
-            acc += reinterpret_cast<const float*>(inbox)[(src * rows_per + rr) * T + tt];
-          reinterpret_cast<uint16_t*>(y)[o] = float_to_bf16_bits(acc * alpha[j]);
-        } else {
-          int32_t acc = 0;
-          for (int src = 0; src < S; ++src)
-            acc += reinterpret_cast<const int32_t*>(inbox)[(src * rows_per + rr) * T + tt];
-          reinterpret_cast<float*>(y)[o] = static_cast<float>(static_cast<double>(acc) * bt * gamma[m] / 128.0);
-          if (acc_out) acc_out[o] = acc;
+    epilogue_bar();  // tok_scale / row_alpha are written
+    // owner: add the S partials of its rows in rank order, then scale and store;
+    // a thread takes one row and four consecutive tokens (the padded inbox rows
+    // make the 16-byte reads of a warp conflict-free; lanes = consecutive rows,
+    // so each output store of a warp is contiguous)
+    if (mbar_wait(smem_u32(&inbox_bar), 0, kWhereGemmEpilogue)) {
+      for (int e = et; e < rows_per * (T / 4); e += 128) {
+        const int rr = e % rows_per, tq = e / rows_per;
+        const int j = w0 + static_cast<int>(rank) * rows_per + rr;
+        if (j >= N) continue;
+        uint32_t sum[4] = {0u, 0u, 0u, 0u};
+        float fsum[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int src = 0; src < S; ++src) {
+          const uint4 v = *reinterpret_cast<const uint4*>(inbox + ((src * rows_per + rr) * IN_STRIDE + 4 * tq) * 4);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (KIND == 0)
+              fsum[i] += __uint_as_float(w[i]);
+            else
+              sum[i] += w[i];  // two's complement: exact int32 sum
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tt = 4 * tq + i, m = t0 + tt;
+          if (m >= M) continue;
+          const int64_t o = static_cast<int64_t>(m) * N + j;
+          if (KIND == 0) {
+            reinterpret_cast<uint16_t*>(y)[o] = float_to_bf16_bits(fsum[i] * row_alpha[rr]);
+          } else {
+            const int32_t acc = static_cast<int32_t>(sum[i]);
+            reinterpret_cast<float*>(y)[o] = w1a8_output(acc, tok_scale[tt]);
+            if (acc_out) acc_out[o] = acc;
+          }
         }
       }
     }
   } else if (warp >= 4) {
     // ---------------- epilogue ----------------
-    // Accumulators -> scaled outputs -> staging tile [T tokens][ROWS] in
-    // shared memory; the accumulators are released as soon as they are read,
-    // then one bulk tensor store writes the tile (rows/tokens past N/M are
-    // clipped by the store). Without an aligned output (N % 8 for bf16,
-    // N % 4 for fp32), or when the tile is too large to stage, the outputs
-    // are stored directly instead.
-    const int q = warp & 3;
+    // Accumulators -> scaled outputs -> staging tile [T tokens][STAGE_COLS]
+    // in shared memory -> one bulk tensor store per staged group of rows
+    // (rows/tokens past N/M are clipped by the store). The accumulators are
+    // released as soon as the last of them is read. Without an aligned
+    // output (N % 8 for bf16, N % 4 for fp32) the outputs are stored
+    // directly instead. The per-row alpha and per-token scale are read once
+    // per tile into registers / shared memory, never per element.
+    constexpr int BLK_PER_GROUP = C::STAGE_COLS / 128;
+    const int q = warp & 3, et = threadIdx.x - 128;
     uint8_t* stage_out = bits_ring + C::SB * C::BITS_BYTES;
+    const bool staged = C::STAGE_OUT && use_tma_store;
     const bool leader = (warp == 4 && lane == 0);
     uint32_t tcount = 0;
     double bt = 0.0;
     if (KIND == 1) bt = static_cast<double>(*beta);
     for (int tile = tile_first; tile < num_tiles; tile += tile_step, ++tcount) {
       const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
-      if (!mbar_wait(smem_u32(&d_full), tcount & 1, kWhereGemmEpilogue)) break;
-      tc_fence_after_sync();
-      if (C::STAGE_OUT && use_tma_store) {
-        if (leader) bulk_wait_read0();  // the previous tile's store has read the staging tile
-        epilogue_bar();
+      if (KIND == 1) {
+        epilogue_bar();  // the previous tile's readers of tok_scale are done
+        for (int tt = et; tt < T; tt += 128)
+          tok_scale[tt] = w1a8_token_scale(bt, t0 + tt < M ? gamma[t0 + tt] : 0.0);
       }
-#pragma unroll 1
-      for (int blk = 0; blk < NB; ++blk) {
-        const int jl = blk * 128 + q * 32 + lane;  // row of the tile = output channel w0 + jl
-        const int j = w0 + jl;
-        const bool jv = j < N;
-        float aj = 0.f;
-        if (KIND == 0 && jv) aj = alpha[j];
-#pragma unroll 1
-        for (int cc = 0; cc < T / 32; ++cc) {
-          uint32_t r[32];
-          __syncwarp();
-          tmem_ld_32x32b_x32(tmem + blk * T + cc * 32 + (static_cast<uint32_t>(q * 32) << 16), r);
-          tmem_wait_ld();
-          if (blk == NB - 1 && cc == T / 32 - 1) {
-            // every accumulator column of this tile has been read: free them
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&d_empty));
-          }
-          const int ml0 = cc * 32;
+      float aj[NB];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int m = t0 + ml0 + i;
+      for (int blk = 0; blk < NB; ++blk) {
+        const int j = w0 + blk * 128 + q * 32 + lane;
+        aj[blk] = (KIND == 0 && j < N) ? alpha[j] : 0.f;
+      }
+      // all four warps leave together if the accumulators never arrive
+      if (!epilogue_bar_and(mbar_wait(smem_u32(&d_full), tcount & 1, kWhereGemmEpilogue))) break;
+      tc_fence_after_sync();
+#pragma unroll 1
+      for (int g = 0; g < NB / BLK_PER_GROUP; ++g) {
+        if (staged && leader) bulk_wait_read0();  // the previous store has read the staging tile
+        epilogue_bar();                           // (and tok_scale is written)
+#pragma unroll 1
+        for (int b = 0; b < BLK_PER_GROUP; ++b) {
+          const int blk = g * BLK_PER_GROUP + b;
+          const int jl = blk * 128 + q * 32 + lane;  // row of the tile = output channel w0 + jl
+          const int js = b * 128 + q * 32 + lane;    // column in the staging tile
+          const int j = w0 + jl;
+          const bool jv = j < N;
+          const float a = (NB == 1 || blk == 0) ? aj[0] : aj[NB - 1];
+#pragma unroll 1
+          for (int cc = 0; cc < T / 32; ++cc) {
+            uint32_t r[32];
+            __syncwarp();
+            tmem_ld_32x32b_x32(tmem + blk * T + cc * 32 + (static_cast<uint32_t>(q * 32) << 16), r);
+            tmem_wait_ld();
+            if (blk == NB - 1 && cc == T / 32 - 1) {
+              // every accumulator column of this tile has been read: free them
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&d_empty));
+            }
+            const int ml0 = cc * 32;
             if (KIND == 0) {
-              const uint16_t v = float_to_bf16_bits(__uint_as_float(r[i]) * aj);
-              if (C::STAGE_OUT && use_tma_store)
-                reinterpret_cast<uint16_t*>(stage_out)[(ml0 + i) * ROWS + jl] = v;
-              else if (jv && m < M)
-                reinterpret_cast<uint16_t*>(y)[static_cast<int64_t>(m) * N + j] = v;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int m = t0 + ml0 + i;
+                const uint16_t v = float_to_bf16_bits(__uint_as_float(r[i]) * a);
+                if (staged)
+                  reinterpret_cast<uint16_t*>(stage_out)[(ml0 + i) * C::STAGE_COLS + js] = v;
+                else if (jv && m < M)
+                  reinterpret_cast<uint16_t*>(y)[static_cast<int64_t>(m) * N + j] = v;
+              }
             } else {
-              const int32_t acc = static_cast<int32_t>(r[i]);
-              const double gm = m < M ? gamma[m] : 0.0;
-              const float v = static_cast<float>(static_cast<double>(acc) * bt * gm / 128.0);
-              if (C::STAGE_OUT && use_tma_store)
-                reinterpret_cast<float*>(stage_out)[(ml0 + i) * ROWS + jl] = v;
-              else if (jv && m < M)
-                reinterpret_cast<float*>(y)[static_cast<int64_t>(m) * N + j] = v;
-              if (acc_out && jv && m < M) acc_out[static_cast<int64_t>(m) * N + j] = acc;
+              // the fp32 form covers the chunk unless some |acc| is very large
+              // (K beyond ~33k); the test is made once per chunk, so the
+              // element loop stays free of branches
+              bool fast = true;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) fast &= w1a8_fast_ok(static_cast<int32_t>(r[i]));
+              float v[32];
+              if (__all_sync(0xffffffffu, fast)) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = w1a8_output_fast(static_cast<int32_t>(r[i]), tok_scale[ml0 + i]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = w1a8_output(static_cast<int32_t>(r[i]), tok_scale[ml0 + i]);
+              }
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int m = t0 + ml0 + i;
+                if (staged)
+                  reinterpret_cast<float*>(stage_out)[(ml0 + i) * C::STAGE_COLS + js] = v[i];
+                else if (jv && m < M)
+                  reinterpret_cast<float*>(y)[static_cast<int64_t>(m) * N + j] = v[i];
+                if (acc_out && jv && m < M) acc_out[static_cast<int64_t>(m) * N + j] = static_cast<int32_t>(r[i]);
+              }
             }
           }
         }
-      }
-      if (C::STAGE_OUT && use_tma_store) {
-        fence_proxy_async_smem();  // staging writes -> visible to the bulk store
-        epilogue_bar();
-        if (leader) {
-          tma_store_2d(&tm_y, smem_u32(stage_out), w0, t0);
-          bulk_commit();
+        if (staged) {
+          fence_proxy_async_smem();  // staging writes -> visible to the bulk store
+          epilogue_bar();
+          if (leader) {
+            tma_store_2d(&tm_y, smem_u32(stage_out), w0 + g * C::STAGE_COLS, t0);
+            bulk_commit();
+          }
         }
       }
     }
-    if (C::STAGE_OUT && use_tma_store && leader) bulk_wait0();
+    if (staged && leader) bulk_wait0();
   }
 
   if (SPLIT && !(warp >= 4 && warp < 8))
