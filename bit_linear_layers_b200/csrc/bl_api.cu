@@ -263,7 +263,7 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
   if (!xq_in) {
     int8_t* xq_ws = static_cast<int8_t*>(ws);
     double* g_ws = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(size_t(M * K)));
-    ln_quant_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, K, xq_ws, g_ws);
+    ln_quant_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
     if ((rc = launch_status()) != BL_OK) return rc;
     codes = xq_ws;
     gam = g_ws;

@@ -54,10 +54,12 @@ template <int KIND, int NB, int T, bool SPLIT>
 struct TsCfg {
   static constexpr int ROWS = 128 * NB;                         // weight rows per tile
   static constexpr int ELEM = KIND == 0 ? 2 : 1;                // activation bytes
-  // pipeline unit: one 128-byte swizzle atom of every activation row
-  static constexpr int UNIT_K = 128 / ELEM;                     // 64 (bf16) or 128 (int8)
-  static constexpr int UPB = ELEM;                              // units per 128-k sign stage
-  static constexpr int X_UNIT_BYTES = T * 128;
+  // pipeline unit: one 128-k sign stage; its activations are ATOMS 128-byte
+  // swizzle atoms of every token row (64 k each for bf16, 128 k for int8)
+  static constexpr int ATOM_K = 128 / ELEM;
+  static constexpr int ATOMS = kTsStageK / ATOM_K;              // 2 (bf16) or 1 (int8)
+  static constexpr int ATOM_BYTES = T * 128;
+  static constexpr int X_UNIT_BYTES = ATOMS * ATOM_BYTES;
   static constexpr int BITS_BYTES = ROWS * 16;                  // one 128-k sign stage
   static constexpr int SB = 4;                                  // sign stages in shared memory
   static constexpr int OUT_ELEM = KIND == 0 ? 2 : 4;            // y element bytes
@@ -71,20 +73,20 @@ struct TsCfg {
   static constexpr int IN_STRIDE = T + 4;
   // staged output [T][STAGE_COLS], or the split-K inbox [S][ROWS/S][IN_STRIDE] of 4-byte partials
   static constexpr int OUT_BYTES = SPLIT ? ROWS * IN_STRIDE * 4 : (STAGE_OUT ? STAGE_COLS * T * OUT_ELEM : 0);
-  static constexpr int SX_FIT = (210 * 1024 - OUT_BYTES - SB * BITS_BYTES) / X_UNIT_BYTES;
+  static constexpr int SX_FIT = (220 * 1024 - OUT_BYTES - SB * BITS_BYTES) / X_UNIT_BYTES;
   static constexpr int SX = SX_FIT > 8 ? 8 : SX_FIT;           // activation units in flight
   static constexpr int X_RING = SX * X_UNIT_BYTES;
   static constexpr int SMEM_BYTES = X_RING + SB * BITS_BYTES + OUT_BYTES + 1024;
-  static constexpr int MMA_K = KIND == 0 ? 16 : 32;             // elements per MMA
-  static constexpr int KSTEPS = 4;                              // MMAs per block per unit (32 B each)
-  static constexpr int A_COLS = 32;                             // TMEM columns per block per unit
-  static constexpr int CH = UNIT_K / 16;                        // 16-bit sign chunks per unit
+  static constexpr int KSTEPS = 4 * ATOMS;                      // MMAs per block per unit (32 bytes of k each)
+  static constexpr int A_COLS = 32 * ATOMS;                     // TMEM columns per block per unit
+  static constexpr int CH = kTsStageK / 16;                     // 16-bit sign chunks per unit (8)
+  static constexpr int COLS_PER_CH = A_COLS / CH;               // 8 (bf16) or 4 (int8)
   static constexpr int D_COLS = NB * T;                         // accumulators
   static constexpr int SA_MAX = (512 - D_COLS) / (NB * A_COLS);
   static constexpr int SA = SA_MAX > 8 ? 8 : SA_MAX;            // sign units in TMEM
   static_assert(SA >= 2, "need at least two sign units");
   static_assert(SX >= 2, "need at least two activation units");
-  static_assert(X_UNIT_BYTES % 1024 == 0 && BITS_BYTES % 1024 == 0, "swizzle alignment");
+  static_assert(ATOM_BYTES % 1024 == 0 && BITS_BYTES % 1024 == 0, "swizzle alignment");
   static_assert(NB == 1 || NB == 2, "one or two 128-row blocks per tile");
 };
 
@@ -112,6 +114,16 @@ __device__ __forceinline__ void tmem_st_32x32b<16>(uint32_t taddr, const uint32_
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// N consecutive 32-bit columns of this warp's lane quarter (N = 16, 32 or 64)
+template <int N>
+__device__ __forceinline__ void tmem_st_wide(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 64) {
+    tmem_st_32x32b<32>(taddr, r);
+    tmem_st_32x32b<32>(taddr + 32, r + 32);
+  } else {
+    tmem_st_32x32b<N>(taddr, r);
+  }
+}
 
 // bulk tensor store of a shared-memory tile (no multicast), tracked by bulk groups
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t c0, int32_t c1) {
@@ -254,8 +266,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
   const int kb_per = (num_kb + S - 1) / S;
   const int kb_first = SPLIT ? static_cast<int>(rank) * kb_per : 0;
   const int kb_last = SPLIT ? min(num_kb, kb_first + kb_per) : num_kb;
-  // pipeline units of this CTA within each tile (whole sign stages)
-  const int u_first = kb_first * C::UPB, u_last = kb_last * C::UPB;
+  // pipeline units (128-k sign stages) of this CTA within each tile
+  const int u_first = kb_first, u_last = kb_last;
   uint8_t* const bits_ring = smem + C::X_RING;
 
   if (threadIdx.x == 0) {
@@ -292,25 +304,22 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
-    // per unit: the sign stage (every UPB units) first, the expanders need
-    // only those; then the activation atom the MMA reads
+    // per unit: the sign stage first (the expanders need only that), then the
+    // unit's activation atoms, all counted on one barrier
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
       for (int tile = tile_first; tile < num_tiles && ok; tile += tile_step) {
         const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
         for (int u = u_first; u < u_last; ++u, ++it) {
-          if (it % C::UPB == 0) {
-            const uint32_t bit_it = it / C::UPB, bs = bit_it % C::SB;
-            if (bit_it >= C::SB &&
-                !mbar_wait(smem_u32(&b_empty[bs]), ((bit_it / C::SB) - 1) & 1, kWhereGemmProducer)) {
-              ok = false;
-              break;
-            }
-            const uint32_t bb = smem_u32(&b_full[bs]);
-            mbar_arrive_expect_tx(bb, C::BITS_BYTES);
-            tma_load_2d(smem_u32(bits_ring + bs * C::BITS_BYTES), &tm_bits, bb, (u / C::UPB) * 4, w0);
+          const uint32_t bs = it % C::SB;
+          if (it >= C::SB && !mbar_wait(smem_u32(&b_empty[bs]), ((it / C::SB) - 1) & 1, kWhereGemmProducer)) {
+            ok = false;
+            break;
           }
+          const uint32_t bb = smem_u32(&b_full[bs]);
+          mbar_arrive_expect_tx(bb, C::BITS_BYTES);
+          tma_load_2d(smem_u32(bits_ring + bs * C::BITS_BYTES), &tm_bits, bb, u * 4, w0);
           const uint32_t xs = it % SX;
           if (it >= SX && !mbar_wait(smem_u32(&x_empty[xs]), ((it / SX) - 1) & 1, kWhereGemmProducer)) {
             ok = false;
@@ -318,12 +327,19 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
           }
           const uint32_t fb = smem_u32(&x_full[xs]);
           mbar_arrive_expect_tx(fb, C::X_UNIT_BYTES);
-          tma_load_2d(smem_u32(smem + xs * C::X_UNIT_BYTES), &tm_x, fb, u * C::UNIT_K, t0);
+#pragma unroll
+          for (int h = 0; h < C::ATOMS; ++h)
+            tma_load_2d(smem_u32(smem + xs * C::X_UNIT_BYTES + h * C::ATOM_BYTES), &tm_x, fb,
+                        u * kTsStageK + h * C::ATOM_K, t0);
         }
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // One barrier per unit: a_full completes once the signs are in tensor
+    // memory and (through the expander that waited for them) the activations
+    // are in shared memory. Every mbarrier test the issuing thread makes holds
+    // up its next MMA by ~100 ns, so it makes exactly one per unit.
     if (lane == 0) {
       const uint32_t idesc = KIND == 0 ? idesc_bf16_f32(128, T) : idesc_s8_s32(128, T);
       uint32_t it = 0, tcount = 0;
@@ -333,28 +349,31 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
         tc_fence_after_sync();
         for (int u = u_first; u < u_last; ++u, ++it) {
           const uint32_t xs = it % SX, a = it % SA;
-          if (!mbar_wait(smem_u32(&x_full[xs]), (it / SX) & 1, kWhereGemmMma) ||
-              !mbar_wait(smem_u32(&a_full[a]), (it / SA) & 1, kWhereGemmMma)) {
+          if (!mbar_wait(smem_u32(&a_full[a]), (it / SA) & 1, kWhereGemmMma)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          // descriptor of the atom's first 32-byte K slice; later slices add
+          // descriptor of each atom's first 32-byte k slice; later slices add
           // their byte offset >> 4 to the start-address field (never carries:
           // the ring lies inside the 256 KB window of the 14-bit field)
-          const uint64_t bd0 = sw128_kmajor_desc(smem_u32(smem + xs * C::X_UNIT_BYTES));
           const uint32_t a_tm0 = a_base + (a * NB) * C::A_COLS;
 #pragma unroll
-          for (int kk = 0; kk < C::KSTEPS; ++kk) {
-            const uint64_t bd = bd0 + static_cast<uint64_t>((kk * 32) >> 4);
-            const uint32_t accum = (u > u_first || kk > 0) ? 1u : 0u;
+          for (int h = 0; h < C::ATOMS; ++h) {
+            const uint64_t bd0 = sw128_kmajor_desc(smem_u32(smem + xs * C::X_UNIT_BYTES + h * C::ATOM_BYTES));
 #pragma unroll
-            for (int blk = 0; blk < NB; ++blk) {
-              const uint32_t a_tm = a_tm0 + blk * C::A_COLS + kk * 8;
-              if (KIND == 0)
-                umma_ts_bf16(tmem + blk * T, a_tm, bd, idesc, accum);
-              else
-                umma_ts_i8(tmem + blk * T, a_tm, bd, idesc, accum);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int kk = h * 4 + k4;
+              const uint64_t bd = bd0 + static_cast<uint64_t>((k4 * 32) >> 4);
+              const uint32_t accum = (u > u_first || kk > 0) ? 1u : 0u;
+#pragma unroll
+              for (int blk = 0; blk < NB; ++blk) {
+                const uint32_t a_tm = a_tm0 + blk * C::A_COLS + kk * 8;
+                if (KIND == 0)
+                  umma_ts_bf16(tmem + blk * T, a_tm, bd, idesc, accum);
+                else
+                  umma_ts_i8(tmem + blk * T, a_tm, bd, idesc, accum);
+              }
             }
           }
           umma_commit(smem_u32(&x_empty[xs]));
@@ -368,57 +387,67 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     // ---------------- sign expanders ----------------
     // With two blocks, warp 8 + 4*b + q expands block b, lane quarter q, all
     // CH chunks of the unit; with one block the two warps of a lane quarter
-    // take half of the chunks each. A unit's signs are 16-bit chunks
-    // g = h*CH + j of the 128-bit stage row (h = unit within the stage).
+    // take half of the chunks each. Chunk g of a unit = bits 16g..16g+15 of
+    // the row's 128-bit sign stage. The expander of rank it % 8 also waits
+    // for the unit's activations before it arrives, so that a_full alone
+    // tells the MMA issuer the unit is ready.
     const int q = warp & 3, part = (warp - 8) >> 2;
     const int blk = NB == 2 ? part : 0;
     constexpr int MY_CH = NB == 2 ? C::CH : C::CH / 2;      // chunks this warp expands
-    constexpr int COLS_PER_CH = C::A_COLS / C::CH;           // 8 (bf16) or 4 (int8)
+    constexpr int COLS_PER_CH = C::COLS_PER_CH;
     const int ch0 = NB == 2 ? 0 : part * MY_CH;
     const int r = blk * 128 + q * 32 + lane;  // sign row within the tile = TMEM lane in its block
-    uint32_t it = 0;
-    bool ok = true;
-    for (int tile = tile_first; tile < num_tiles && ok; tile += tile_step) {
-      for (int u = u_first; u < u_last; ++u, ++it) {
-        const uint32_t a = it % SA, bit_it = it / C::UPB, bs = bit_it % C::SB;
-        if ((it >= SA && !mbar_wait(smem_u32(&a_empty[a]), ((it / SA) - 1) & 1, kWhereGemmExpander)) ||
-            !mbar_wait(smem_u32(&b_full[bs]), (bit_it / C::SB) & 1, kWhereGemmExpander)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const uint4 wv = *reinterpret_cast<const uint4*>(bits_ring + bs * C::BITS_BYTES + r * 16);
-        const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-        const int h = static_cast<int>(it % C::UPB);
-        const uint32_t taddr = a_base + (a * NB + blk) * C::A_COLS + ch0 * COLS_PER_CH +
-                               (static_cast<uint32_t>(q * 32) << 16);
-        // this warp's chunks are words off_w .. off_w + MY_CH/2 - 1 of the row
-        constexpr int MY_W = MY_CH / 2;
-        const int off_w = (h * C::CH + ch0) >> 1;  // even chunk offset
-        uint32_t seg[MY_W];
+    // The expanders see only a flat sequence of units (ring slots). Software
+    // pipelined: the store of unit `it` is in flight while the warp waits for
+    // the inputs of unit it + 1; only then is unit `it` signalled.
+    const int my_tiles = tile_first < num_tiles ? (num_tiles - tile_first + tile_step - 1) / tile_step : 0;
+    const uint32_t total = static_cast<uint32_t>(my_tiles * (u_last - u_first));
+    uint32_t v[MY_CH * COLS_PER_CH];
+    auto inputs_ready = [&](uint32_t it) -> bool {
+      const uint32_t a = it % SA, bs = it % C::SB;
+      const bool ok = (it < static_cast<uint32_t>(SA) ||
+                       mbar_wait(smem_u32(&a_empty[a]), ((it / SA) - 1) & 1, kWhereGemmExpander)) &&
+                      mbar_wait(smem_u32(&b_full[bs]), (it / C::SB) & 1, kWhereGemmExpander);
+      return __all_sync(0xffffffffu, ok);
+    };
+    auto expand_and_store = [&](uint32_t it) {
+      tc_fence_after_sync();
+      const uint32_t a = it % SA, bs = it % C::SB;
+      const uint4 wv = *reinterpret_cast<const uint4*>(bits_ring + bs * C::BITS_BYTES + r * 16);
+      const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+      const uint32_t taddr = a_base + (a * NB + blk) * C::A_COLS + ch0 * COLS_PER_CH +
+                             (static_cast<uint32_t>(q * 32) << 16);
+      // this warp's chunks are words ch0/2 .. ch0/2 + MY_CH/2 - 1 of the row
 #pragma unroll
-        for (int w = 0; w < MY_W; ++w) {
-          const int idx = off_w + w;
-          seg[w] = idx == 0 ? wd[0] : idx == 1 ? wd[1] : idx == 2 ? wd[2] : wd[3];
-        }
-        uint32_t v[MY_CH * COLS_PER_CH];
-#pragma unroll
-        for (int j = 0; j < MY_CH; ++j) {
-          const uint32_t chunk = (seg[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-          if (KIND == 0)
-            expand16_bf16(chunk, v + j * COLS_PER_CH);
-          else
-            expand16_i8(chunk, v + j * COLS_PER_CH);
-        }
-        tmem_st_32x32b<MY_CH * COLS_PER_CH>(taddr, v);
-        tmem_wait_st();
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(smem_u32(&a_full[a]));
-          if (it % C::UPB == C::UPB - 1) mbar_arrive(smem_u32(&b_empty[bs]));
-        }
+      for (int j = 0; j < MY_CH; ++j) {
+        const uint32_t word = NB == 2 ? wd[j >> 1] : (ch0 == 0 ? wd[j >> 1] : wd[2 + (j >> 1)]);
+        const uint32_t chunk = (word >> (16 * (j & 1))) & 0xFFFFu;  // ch0 is even
+        if (KIND == 0)
+          expand16_bf16(chunk, v + j * COLS_PER_CH);
+        else
+          expand16_i8(chunk, v + j * COLS_PER_CH);
       }
+      tmem_st_wide<MY_CH * COLS_PER_CH>(taddr, v);
+    };
+    bool ok = total > 0 && inputs_ready(0);
+    if (ok) expand_and_store(0);
+    for (uint32_t it = 0; ok && it < total; ++it) {
+      const bool more = it + 1 < total;
+      const bool next_ok = !more || inputs_ready(it + 1);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        // the expander of rank it % 8 also waits for the unit's activations
+        const bool x_waiter = (warp - 8) == static_cast<int>(it % kTsExpanders);
+        if (x_waiter && !mbar_wait(smem_u32(&x_full[it % SX]), (it / SX) & 1, kWhereGemmExpander))
+          ok = false;  // a_full then never completes: the MMA issuer gives up on its own bounded wait
+        else
+          mbar_arrive(smem_u32(&a_full[it % SA]));
+        mbar_arrive(smem_u32(&b_empty[it % C::SB]));
+      }
+      ok = (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0) && next_ok;
+      if (ok && more) expand_and_store(it + 1);
     }
   } else if (warp >= 4 && SPLIT) {
     // ---------------- split-K epilogue: push partials, owner reduces ----------------

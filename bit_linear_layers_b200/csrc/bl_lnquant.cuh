@@ -2,104 +2,150 @@
 // ("BitNet b1.58" page, section 1: LN of Eq.(8), then Eq.(4)-(5) with
 // Q_b = 128). One CTA per token.
 //
-// Statistics are fp64: the sum of bf16 values is exact in fp64 (their
-// exponent span is far below 53 bits), so mu = sum/K is the same correctly
-// rounded double the CPU statement gets; var, sqrt(var + eps) and
-// gamma = max|x - mu| / sqrt(var + eps) follow in fp64 (max of |(x-mu)/s|
-// equals max|x-mu| / s because rounded division by s > 0 is monotonic).
+// Statistics are fp64: the sum of bf16 values is exact in fp64 whenever their
+// exponents span less than ~40 binades (any realistic activation row), so
+// mu = sum/K is the same correctly rounded double the CPU statement gets;
+// var = sum (x - mu)^2 / K, root = sqrt(var + eps) follow in fp64.
+// max_k |x_k - mu| is taken as max(x_max - mu, mu - x_min) in fp64: the
+// rounded difference is monotonic in x, so this is exactly the largest
+// rounded |x_k - mu|; and gamma = max|x - mu| / root equals max |(x - mu)/root|
+// because rounded division by root > 0 is monotonic.
 //
-// The code q = clamp(rint(ln * 128 / gamma), -127, 127) is decided as in
-// fp64. Fast path: v32 = fp32(x - mu) * fp32(128 / max|x-mu|), within
-// 3.1 * 2^-24 * 128 < 2.5e-5 of the exact value, and the fp64 value is within
-// ~1e-13 of exact; so whenever v32 is farther than 1e-4 from a half-integer
-// both round to the same integer. Otherwise the fp64 steps are evaluated in
-// the order of the formula. gamma == 0 (constant token) gives all-zero codes.
+// The code q = clamp(rint(ln * 128 / gamma), -127, 127), whose exact value is
+// (x - mu) * 128 / max|x - mu|, is decided as in fp64. Fast path, all fp32:
+// d32 = (x - mu_hi) - mu_lo with mu = mu_hi + mu_lo to ~2^-48, times
+// c32 = fp32(128 / max|x - mu|); each of the four roundings moves the value by
+// at most 128 * 2^-24 (bf16 inputs that are not all equal differ by at least
+// one bf16 ulp, which keeps |mu| / max|x - mu| below ~2^9, so neither the
+// split of mu nor |x - mu_hi| > |x - mu| adds anything measurable), so v32
+// lies within 3.1e-5 of the exact value, and the
+// fp64 evaluation within ~1e-13 of it: whenever v32 is farther than 1e-4 from
+// a half-integer both round to the same integer. Otherwise the fp64 steps are
+// evaluated in the order of the formula. max|x - mu| == 0 (constant token)
+// gives gamma = 0 and all-zero codes.
 #pragma once
 
 #include "bl_common.cuh"
 
 namespace bl {
 
-constexpr int kLnThreads = 256;
+constexpr int kLnThreads = 256;  // one CTA per token
+constexpr int kLnWarps = kLnThreads / 32;
 constexpr double kLnEps = 1e-5;
 
-template <typename T, typename Op>
-__device__ __forceinline__ T block_reduce(T v, T* sh, Op op) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();  // sh may still be read from a previous reduction
-  if (lane == 0) sh[warp] = v;
-  __syncthreads();
-  v = sh[0];
-#pragma unroll
-  for (int w = 1; w < kLnThreads / 32; ++w) v = op(v, sh[w]);
-  return v;
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// bf16 bits -> the same value as a double, built with integer operations
+// (the float -> double conversion unit is the slowest pipe of this kernel):
+// for a normal bf16 the double's high word is the sign, the exponent
+// rebiased by 1023 - 127 = 896 and the 7 mantissa bits; its low word is 0.
+// Zeros, subnormals, infinities and NaNs take the conversion instruction.
+__device__ __forceinline__ double bf16_to_double(uint32_t b16) {
+  const uint32_t e = b16 & 0x7F80u;
+  if (e == 0u || e == 0x7F80u) return static_cast<double>(__uint_as_float(b16 << 16));
+  const uint32_t hi = ((b16 & 0x8000u) << 16) | (((b16 & 0x7FFFu) << 13) + (896u << 20));
+  return __hiloint2double(static_cast<int>(hi), 0);
 }
 
-struct SumOp {
-  __device__ double operator()(double a, double b) const { return a + b; }
-};
-struct MaxOp {
-  __device__ double operator()(double a, double b) const { return a > b ? a : b; }
-};
-
-__device__ __forceinline__ int quant_code(float xv, double mu, double root, double gamma,
-                                          float c32) {
+// exact fp64 evaluation of the code, in the order of the formula
+__device__ __noinline__ int quant_code_exact(float xv, double mu, double root, double gamma) {
   const double d = static_cast<double>(xv) - mu;
-  const float v32 = static_cast<float>(d) * c32;
-  const float frac = v32 - floorf(v32);
-  float r;
-  if (fabsf(frac - 0.5f) > 1e-4f) {
-    r = rintf(v32);
-  } else {
-    const double ln = d / root;
-    const double v = ln * 128.0 / gamma;
-    r = static_cast<float>(rint(v));
-  }
-  r = fminf(fmaxf(r, -127.f), 127.f);
-  return static_cast<int>(r);
+  const double ln = d / root;
+  const double v = ln * 128.0 / gamma;
+  return static_cast<int>(fmin(fmax(rint(v), -127.0), 127.0));
 }
 
-__global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __restrict__ x,
+struct LnQuantParams {
+  float mu_hi, mu_lo, c32;
+  double mu, root, gamma;
+};
+
+__device__ __forceinline__ int quant_code(float xv, const LnQuantParams& p) {
+  const float d32 = (xv - p.mu_hi) - p.mu_lo;
+  const float v32 = d32 * p.c32;
+  const float frac = v32 - floorf(v32);
+  if (fabsf(frac - 0.5f) <= 1e-4f) return quant_code_exact(xv, p.mu, p.root, p.gamma);
+  return static_cast<int>(fminf(fmaxf(rintf(v32), -127.f), 127.f));
+}
+
+// CTA-wide sum (fp64) of one value per thread; every thread gets the total
+__device__ __forceinline__ double ln_block_sum(double v, double* sh) {
+  v = warp_sum(v);
+  __syncthreads();  // sh may still be read from a previous reduction
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+  __syncthreads();
+  double t = sh[0];
+#pragma unroll
+  for (int w = 1; w < kLnWarps; ++w) t += sh[w];
+  return t;
+}
+
+__global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                               int64_t K, int8_t* __restrict__ xq,
                                                               double* __restrict__ gamma_out) {
-  __shared__ double sh[kLnThreads / 32];
+  __shared__ double sh[kLnWarps];
+  __shared__ float shm[2][kLnWarps];
   const int64_t m = blockIdx.x;
+  if (m >= M) return;  // uniform per CTA
   const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
   const int64_t nvec = K / 8;  // 8 bf16 per 16-byte load
 
-  double s = 0.0;
-  for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
-    const uint4 v = row[i];
-    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      s += static_cast<double>(__uint_as_float(h[j] << 16)) +
-           static_cast<double>(__uint_as_float(h[j] & 0xFFFF0000u));
-  }
-  s = block_reduce(s, sh, SumOp{});
-  const double mu = s / static_cast<double>(K);
-
-  double sq = 0.0, dmax = 0.0;
+  // pass 1: fp64 sum (two chains), fp32 max and min
+  double s0 = 0.0, s1 = 0.0;
+  float xmax = -INFINITY, xmin = INFINITY;
   for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
     const uint4 v = row[i];
     const uint32_t h[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const double d0 = static_cast<double>(__uint_as_float(h[j] << 16)) - mu;
-      const double d1 = static_cast<double>(__uint_as_float(h[j] & 0xFFFF0000u)) - mu;
-      sq += d0 * d0 + d1 * d1;
-      dmax = fmax(dmax, fmax(fabs(d0), fabs(d1)));
+      s0 += bf16_to_double(h[j] & 0xFFFFu);
+      s1 += bf16_to_double(h[j] >> 16);
+      const float a = bf16_lo(h[j]), b = bf16_hi(h[j]);
+      xmax = fmaxf(xmax, fmaxf(a, b));
+      xmin = fminf(xmin, fminf(a, b));
     }
   }
-  sq = block_reduce(sq, sh, SumOp{});
-  dmax = block_reduce(dmax, sh, MaxOp{});
-  const double root = sqrt(sq / static_cast<double>(K) + kLnEps);
-  const double gamma = dmax / root;
-  if (threadIdx.x == 0) gamma_out[m] = gamma;
+  xmax = warp_max(xmax);
+  xmin = -warp_max(-xmin);
+  if ((threadIdx.x & 31) == 0) {
+    shm[0][threadIdx.x >> 5] = xmax;
+    shm[1][threadIdx.x >> 5] = xmin;
+  }
+  const double mu = ln_block_sum(s0 + s1, sh) / static_cast<double>(K);  // its barriers publish shm
+  xmax = shm[0][0];
+  xmin = shm[1][0];
+#pragma unroll
+  for (int w = 1; w < kLnWarps; ++w) {
+    xmax = fmaxf(xmax, shm[0][w]);
+    xmin = fminf(xmin, shm[1][w]);
+  }
 
-  const float c32 = dmax > 0.0 ? static_cast<float>(128.0 / dmax) : 0.f;
+  // pass 2: sum of squared deviations in fp64
+  double q0 = 0.0, q1 = 0.0;
+  for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
+    const uint4 v = row[i];
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const double d0 = bf16_to_double(h[j] & 0xFFFFu) - mu;
+      const double d1 = bf16_to_double(h[j] >> 16) - mu;
+      q0 = fma(d0, d0, q0);
+      q1 = fma(d1, d1, q1);
+    }
+  }
+  const double sq = ln_block_sum(q0 + q1, sh);
+  const double dmax = fmax(static_cast<double>(xmax) - mu, mu - static_cast<double>(xmin));
+  LnQuantParams p;
+  p.mu = mu;
+  p.root = sqrt(sq / static_cast<double>(K) + kLnEps);
+  p.gamma = dmax / p.root;
+  p.mu_hi = static_cast<float>(mu);
+  p.mu_lo = static_cast<float>(mu - static_cast<double>(p.mu_hi));
+  p.c32 = dmax > 0.0 ? static_cast<float>(128.0 / dmax) : 0.f;
+  if (threadIdx.x == 0) gamma_out[m] = p.gamma;
+
+  // pass 3: codes, 8 per thread per step
   uint2* out = reinterpret_cast<uint2*>(xq + m * K);
   for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
     const uint4 v = row[i];
@@ -108,10 +154,9 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
     if (dmax > 0.0) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int q0 = quant_code(__uint_as_float(h[j] << 16), mu, root, gamma, c32);
-        const int q1 = quant_code(__uint_as_float(h[j] & 0xFFFF0000u), mu, root, gamma, c32);
-        const uint32_t pair = (static_cast<uint32_t>(q0) & 0xFFu) |
-                              ((static_cast<uint32_t>(q1) & 0xFFu) << 8);
+        const int q0c = quant_code(bf16_lo(h[j]), p);
+        const int q1c = quant_code(bf16_hi(h[j]), p);
+        const uint32_t pair = (static_cast<uint32_t>(q0c) & 0xFFu) | ((static_cast<uint32_t>(q1c) & 0xFFu) << 8);
         packed_codes[j >> 1] |= pair << (16 * (j & 1));
       }
     }
