@@ -43,13 +43,15 @@ bool set_smem(Kernel k, int bytes) {
 }
 
 // every tensor-core GEMM configuration the dispatch below can launch
+template <int KIND, int T>
+bool set_ts_smem_t() {
+  return set_smem(gemm_ts_kernel<KIND, 1, T, false>, TsCfg<KIND, 1, T, false>::SMEM_BYTES) &&
+         set_smem(gemm_ts_kernel<KIND, 1, T, true>, TsCfg<KIND, 1, T, true>::SMEM_BYTES);
+}
 template <int KIND>
 bool set_ts_smem() {
   return set_smem(gemm_ts_kernel<KIND, 1, 256, false>, TsCfg<KIND, 1, 256, false>::SMEM_BYTES) &&
-         set_smem(gemm_ts_kernel<KIND, 2, 128, false>, TsCfg<KIND, 2, 128, false>::SMEM_BYTES) &&
-         set_smem(gemm_ts_kernel<KIND, 2, 128, true>, TsCfg<KIND, 2, 128, true>::SMEM_BYTES) &&
-         set_smem(gemm_ts_kernel<KIND, 2, 32, false>, TsCfg<KIND, 2, 32, false>::SMEM_BYTES) &&
-         set_smem(gemm_ts_kernel<KIND, 2, 32, true>, TsCfg<KIND, 2, 32, true>::SMEM_BYTES);
+         set_ts_smem_t<KIND, 128>() && set_ts_smem_t<KIND, 64>() && set_ts_smem_t<KIND, 32>();
 }
 
 int device_setup(int* num_sms) {
@@ -204,39 +206,46 @@ int launch_ts_cfg(const CUtensorMap& tm_x, const CUtensorMap& tm_bits, int64_t M
 }
 
 // activations [M][K] (bf16 for KIND 0, int8 codes for KIND 1) x packed signs [N][K/32].
-// Large bf16 problems: 128-row x 256-token tiles (one 128x256 MMA per K step),
-// persistent. Otherwise (and for int8, whose fp32 output tile would be too large
-// to stage for one bulk store) 256-row tiles of 128 or 32 tokens, split over a
-// cluster along K when the tiles alone would leave SMs idle.
+// Tiles of 128 weight rows. Problems with M >= 256 whose 128-row x 256-token
+// tiles occupy at least half of the SMs use those (one 128x256 MMA per
+// k-step, the most tensor work per instruction). Otherwise tiles of 32, 64 or 128 tokens
+// (the smallest that covers M, up to 128), split over a cluster along K when
+// the tiles alone would leave SMs idle. (Chosen from timings of every
+// configuration on the decode-batch, 1.3B and 7B shapes: 128-row tiles beat
+// 256-row ones, and split-K pays whenever it raises the CTA count.)
+template <int KIND, int T>
+int launch_ts_t(const CUtensorMap& tm_x, const CUtensorMap& tm_bits, int64_t M, int64_t N, int64_t K,
+                const float* alpha, const double* gamma, const float* beta, void* y, int32_t* acc_out,
+                int num_sms, cudaStream_t s) {
+  const int64_t tiles = cdiv(M, T) * cdiv(N, 128);
+  const int S = split_factor(tiles, int(K / kTsStageK), num_sms);
+  return S > 1 ? launch_ts_cfg<KIND, 1, T, true>(tm_x, tm_bits, M, N, K, S, alpha, gamma, beta, y, acc_out, num_sms, s)
+               : launch_ts_cfg<KIND, 1, T, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out, num_sms, s);
+}
+
 template <int KIND>
 int launch_ts(const void* act, const uint32_t* packed, int64_t M, int64_t N, int64_t K,
               const float* alpha, const double* gamma, const float* beta, void* y, int32_t* acc_out,
               int num_sms, cudaStream_t s) {
   const int elem = KIND == 0 ? 2 : 1;
   const CUtensorMapDataType xt = KIND == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  const int num_kb = int(K / kTsStageK);
-  CUtensorMap tm_x, tm_bits;
   const int64_t big_tiles = cdiv(M, 256) * cdiv(N, 128);
-  if (KIND == 0 && M >= 256 && 2 * big_tiles >= num_sms) {
-    if (!make_map_2d(&tm_x, act, xt, elem, uint64_t(K), uint64_t(M), 128 / elem, 256, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4, 128,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
-      return BL_ERR_CUDA;
-    return launch_ts_cfg<KIND, 1, 256, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out,
-                                               num_sms, s);
-  }
-  const int T = M > 32 ? 128 : 32;
+  const int T = (M >= 256 && 2 * big_tiles >= int64_t(num_sms)) ? 256 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
+  CUtensorMap tm_x, tm_bits;
   if (!make_map_2d(&tm_x, act, xt, elem, uint64_t(K), uint64_t(M), 128 / elem, uint32_t(T), CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4, 256,
+      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4, 128,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return BL_ERR_CUDA;
-  const int64_t tiles = cdiv(M, T) * cdiv(N, 256);
-  const int S = split_factor(tiles, num_kb, num_sms);
-  if (T == 128)
-    return S > 1 ? launch_ts_cfg<KIND, 2, 128, true>(tm_x, tm_bits, M, N, K, S, alpha, gamma, beta, y, acc_out, num_sms, s)
-                 : launch_ts_cfg<KIND, 2, 128, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out, num_sms, s);
-  return S > 1 ? launch_ts_cfg<KIND, 2, 32, true>(tm_x, tm_bits, M, N, K, S, alpha, gamma, beta, y, acc_out, num_sms, s)
-               : launch_ts_cfg<KIND, 2, 32, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out, num_sms, s);
+  switch (T) {
+    case 256:
+      return launch_ts_cfg<KIND, 1, 256, false>(tm_x, tm_bits, M, N, K, 1, alpha, gamma, beta, y, acc_out, num_sms, s);
+    case 128:
+      return launch_ts_t<KIND, 128>(tm_x, tm_bits, M, N, K, alpha, gamma, beta, y, acc_out, num_sms, s);
+    case 64:
+      return launch_ts_t<KIND, 64>(tm_x, tm_bits, M, N, K, alpha, gamma, beta, y, acc_out, num_sms, s);
+    default:
+      return launch_ts_t<KIND, 32>(tm_x, tm_bits, M, N, K, alpha, gamma, beta, y, acc_out, num_sms, s);
+  }
 }
 
 // ---- W1A8 shared body -----------------------------------------------------------

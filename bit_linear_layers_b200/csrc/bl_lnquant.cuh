@@ -61,12 +61,18 @@ struct LnQuantParams {
   double mu, root, gamma;
 };
 
+// |v32| <= 128 + 1e-3, so adding 1.5 * 2^23 rounds it to an integer (ties to
+// even) in the float's low mantissa bits: the integer comes out of the bit
+// pattern and v32 - rounded is the distance to it, without the (slow)
+// conversion-unit instructions floor / rint / float-to-int.
 __device__ __forceinline__ int quant_code(float xv, const LnQuantParams& p) {
   const float d32 = (xv - p.mu_hi) - p.mu_lo;
   const float v32 = d32 * p.c32;
-  const float frac = v32 - floorf(v32);
-  if (fabsf(frac - 0.5f) <= 1e-4f) return quant_code_exact(xv, p.mu, p.root, p.gamma);
-  return static_cast<int>(fminf(fmaxf(rintf(v32), -127.f), 127.f));
+  const float big = v32 + 12582912.0f;  // 1.5 * 2^23
+  const float dist = v32 - (big - 12582912.0f);
+  if (fabsf(dist) >= 0.5f - 1e-4f) return quant_code_exact(xv, p.mu, p.root, p.gamma);
+  const int q = __float_as_int(big) - 0x4B400000;
+  return min(max(q, -127), 127);
 }
 
 // CTA-wide sum (fp64) of one value per thread; every thread gets the total

@@ -47,6 +47,8 @@ FULL = [
     (300, 1000, 1024), (1000, 1100, 512),
     # enough tiles for the 128-row x 256-token configuration, ragged in M and N
     (300, 9100, 256),
+    # 64-token tiles split along K; 32-, 64- and 128-token tiles with more tiles than SMs
+    (48, 1000, 512), (20, 20000, 128), (40, 20000, 256), (100, 20000, 256),
 ]
 
 

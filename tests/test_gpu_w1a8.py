@@ -76,7 +76,9 @@ def _run(bl, oracle, M, N, K, seed, kind="laplace_channel", w_mean=0.001, full=T
 FULL = [(4, 256, 256), (1, 128, 128), (7, 200, 384), (16, 129, 256), (17, 300, 512),
         (130, 257, 640), (300, 1000, 1024), (512, 640, 2048),
         # many tiles, ragged in M and N
-        (260, 9500, 128)]
+        (260, 9500, 128),
+        # 64-token tiles split along K; 32-, 64- and 128-token tiles with more tiles than SMs
+        (48, 700, 384), (20, 20000, 128), (40, 20000, 128), (100, 20000, 128)]
 
 
 @pytest.mark.parametrize("M,N,K", FULL)
