@@ -224,6 +224,13 @@ __host__ __device__ constexpr uint32_t idesc_s8_s32(int m, int n) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: wait for the grids this one depends on (a
+// no-op when it was not launched with programmatic serialisation), and let
+// the dependents of this grid be scheduled
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // misc
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
 

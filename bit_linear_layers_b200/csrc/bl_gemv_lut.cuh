@@ -61,8 +61,6 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
                "r"(__float_as_uint(v)), "r"(remote_bar)
                : "memory");
 }
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // NP = pages (16-word groups) per slice; slice_words <= 16 * NP.
 // One-page slices fit two CTAs per SM (registers capped at 128), which lets

@@ -129,7 +129,8 @@ int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* 
  *   gamma_m = max_k |ln_k|
  *   q_mk = clamp(round_half_even(ln_k * 128 / gamma_m), -127, 127)  (0 if gamma_m == 0)
  *   acc[m][j] = sum_k s_jk * q_mk        (exact int32)
- *   y[m][j] = fp32( acc * beta * gamma_m / 128 )   (evaluated in fp64)
+ *   y[m][j] = fp32( acc * beta * gamma_m / 128 )   (the exact value rounded once; within 1 ulp
+ *                                                 of that rounding near rounding midpoints)
  * LN statistics and the quantisation decision are taken in fp64.
  * x [M x K] bf16, packed [N x K/32] (from BL_PACK_BITNET), beta: DEVICE
  * pointer to one float (so pack -> forward needs no host round trip),

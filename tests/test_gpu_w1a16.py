@@ -164,3 +164,33 @@ def test_w1a16_overlap_flag_chain(bl, oracle):
         check_w1a16(bf16_to_f64(y).ravel(), y_ref.ravel(), a, xin, np.zeros(N, dtype=np.int64), js,
                     what=f"layer {i}")
         xin = bf16_bits(y.cpu())
+
+
+@pytest.mark.parametrize("M", [16, 48, 300])
+def test_w1a16_overlap_flag_chain_gemm(bl, M):
+    """BL_FLAG_OVERLAP_PREVIOUS on calls that take the tensor-core path
+    (M > 4, where the flag must not change anything): a chain of dependent
+    calls that ping-pongs between two buffers, so every layer also overwrites
+    the buffer the layer before it read. The results must equal, bit for bit,
+    the same chain run without the flag."""
+    from bit_linear_layers_b200 import synthetic
+    N = K = 1024
+    layers = 6
+    dev = []
+    for i in range(layers):
+        W = synthetic.weights(N, K, 300 + i, device="cuda")
+        dev.append(bl.bin_pack(W, bl.BL_PACK_FBI))
+    x = synthetic.activations(M, K, 11, device="cuda")
+
+    def run(flags):
+        bufs = [x.clone(), torch.empty_like(x)]
+        for i, (p, a) in enumerate(dev):
+            bl.bin_linear_w1a16(bufs[i % 2], p, a, out=bufs[(i + 1) % 2], flags=flags)
+        torch.cuda.synchronize()
+        return bufs[layers % 2].clone()
+
+    ref = run(0)
+    for _ in range(3):
+        got = run(bl.BL_FLAG_OVERLAP_PREVIOUS)
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    assert bl.device_error() == (0, 0)
