@@ -34,6 +34,10 @@ struct DeviceState {
   std::once_flag once;
   int status = BL_ERR_NO_DEVICE;
   int num_sms = 0;
+  // how many clusters of 2 / 4 / 8 tensor-core GEMM CTAs (one CTA per SM)
+  // can be resident at once: clusters must fit inside a GPC, so this is
+  // below num_sms / S (on B200: 74 / 33 / 15)
+  int cluster_cap[9] = {};
 };
 DeviceState g_devices[kMaxDevices];
 
@@ -77,10 +81,39 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
               set_ts_smem<0>() && set_ts_smem<1>();
     if (!ok) cudaGetLastError();
+    for (int S : {2, 4, 8}) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(S), 1, 1);
+      cfg.blockDim = dim3(kTsThreads, 1, 1);
+      cfg.dynamicSmemBytes = TsCfg<0, 1, 128, true>::SMEM_BYTES;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_ts_kernel<0, 1, 128, true>, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = st.num_sms / (2 * S);  // conservative: half of the SMs
+      }
+      st.cluster_cap[S] = n;
+    }
     st.status = ok ? BL_OK : BL_ERR_CUDA;
   });
   if (num_sms) *num_sms = st.num_sms;
   return st.status;
+}
+
+// co-resident cluster capacity of the current device for clusters of S GEMM CTAs
+int cluster_capacity(int S) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 0;
+  }
+  return g_devices[dev].cluster_cap[S];
 }
 
 int launch_status() {
@@ -152,12 +185,13 @@ cudaError_t launch_lut(const uint16_t* x, const uint32_t* packed, const float* a
 // ---- tensor-core GEMM with the signs in tensor memory ------------------------------
 // activations [M][K] (bf16 for KIND 0, int8 codes for KIND 1) x packed signs [N][K/32]
 // Split factor for a problem of `tiles` output tiles and `num_kb` k-blocks:
-// the largest S in {8, 4, 2} (S must divide the 256 rows of a tile) that
-// keeps tiles * S within the SMs and leaves every CTA at least one k-block.
-// Returns 1 when the persistent (unsplit) kernel should be used.
+// the largest S in {8, 4, 2} (S divides the 128 rows of a tile) whose
+// `tiles` clusters of S CTAs are all resident at once (one wave) and that
+// leaves every CTA at least one k-block. Returns 1 when the persistent
+// (unsplit) kernel should be used.
 int split_factor(int64_t tiles, int num_kb, int num_sms) {
   for (int S : {8, 4, 2}) {
-    if (tiles * S > num_sms || S > num_kb) continue;
+    if (tiles * S > num_sms || tiles > cluster_capacity(S) || S > num_kb) continue;
     if (((num_kb + S - 1) / S) * (S - 1) >= num_kb) continue;
     return S;
   }
