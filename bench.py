@@ -349,7 +349,7 @@ class W1A8(Workload):
     dtype = "s8"
     kernel = "ln_quant_kernel + gemm_ts_kernel<1,2,128,*> (one call; time includes LN + quantisation)"
     sources = [CSRC + "bl_gemm_ts.cuh", CSRC + "bl_lnquant.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
-    traffic_file = None
+    traffic_file = "bitlinear_w1a8_1p3b_512tokens.traffic.json"  # the GEMM launches' DRAM bytes
     launches_per_step = 4
     rotate = 16
 
