@@ -214,8 +214,8 @@ class Decode(Workload):
                 W = synthetic.weights(self.N, self.K, seed=2).to(dev)
                 x = synthetic.activations(self.M, self.K, seed=2).to(dev)
             else:       # further seeded draws made on the device
-                W = synthetic.weights(self.N, self.K, seed=2 + 1000 * i + 7 * rank, device=dev)
-                x = synthetic.activations(self.M, self.K, seed=2 + 1000 * i + 7 * rank, device=dev)
+                W = synthetic.weights(self.N, self.K, seed=replica_seed(2, i, rank), device=dev)
+                x = synthetic.activations(self.M, self.K, seed=replica_seed(2, i, rank), device=dev)
             p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
             self.packs.append(p)
             self.alphas.append(a)
@@ -491,11 +491,32 @@ def run_workload(wl, steps, warmup, rank, world, dev, sampler=None):
     del g2
     clocks = sampler.stop() if sampler is not None else None
 
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
     return ms, ms_e2e, clocks
+
+
+def max_over_ranks(times, world, device):
+    """Each rank's device-timed milliseconds -> the maximum over all ranks
+    (every rank takes part; a no-op for one rank)."""
+    if world <= 1:
+        return list(times)
+    import torch
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def replica_seed(base, copy, rank):
+    """Seed of rotating input copy `copy` on `rank`: copy 0 is the seeded
+    workload itself on every rank; the others differ per rank, so replicas
+    do not stream identical weights."""
+    return base if copy == 0 else base + 1000 * copy + 7 * rank
+
+
+def whole_job_value(world, steps, units_per_step, ms, scale):
+    """Aggregate throughput of all ranks: every rank processed `steps`
+    steps of `units_per_step` units in at most `ms` milliseconds."""
+    return world * steps * units_per_step / (ms * 1e-3) / scale
 
 
 def cpu_baseline(wl, target_s=10.0):
@@ -523,8 +544,8 @@ def summarize(wl, ms, ms_e2e, steps, world, peaks, peak_kind):
             else f"fallback ({peak_key})"}
     if isinstance(wl, Decode):
         roof["algorithmic_bytes_per_launch"] = wl.alg_b
-    value = world * steps * wl.units_per_step() / timed_s / wl.scale
-    e2e = {"value": world * steps * wl.units_per_step() / (ms_e2e * 1e-3) / wl.scale, "unit": wl.unit,
+    value = whole_job_value(world, steps, wl.units_per_step(), ms, wl.scale)
+    e2e = {"value": whole_job_value(world, steps, wl.units_per_step(), ms_e2e, wl.scale), "unit": wl.unit,
            "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h, "ms_per_step": ms_e2e / steps}
     return value, roof, e2e
 
