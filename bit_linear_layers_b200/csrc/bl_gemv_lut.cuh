@@ -22,7 +22,8 @@
 //     half-warps visit the four bytes of a word in orders rotated by one, so
 //     each warp's 32 lookups land on 32 distinct banks;
 //   * a warp handles 32 rows as 16 row pairs (half-warp = one row); each lane
-//     reads one packed word per row per 16-word page, prefetched into
+//     reads one packed word per row per 16-word page (its 64 table lookups
+//     are all issued before the adds, for latency overlap), prefetched into
 //     registers before anything else (and before griddepcontrol.wait, so a
 //     launch with programmatic serialisation streams its weights while the
 //     previous kernel finishes);
@@ -148,22 +149,25 @@ __global__ void __launch_bounds__(kLutThreads, NP == 1 ? 2 : 1) gemv_w1a16_lut_k
     colb[s] = (i * 16 + wl) * 4;
     sel[s] = 0x5504u | (i << 4);  // byte0 <- column byte, byte1 <- word byte i, bytes 2,3 <- 0
   }
+  // all 64 lookups of a page are issued before any of them is added, so the
+  // shared-memory latency overlaps (a lane whose word lies past the slice
+  // reads a zero word: its lookups are discarded below)
   float acc[16];
 #pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    float a = 0.f;
+  for (int p = 0; p < 16; ++p) acc[p] = 0.f;
 #pragma unroll
-    for (int pg = 0; pg < NP; ++pg) {
-      if (pg * 16 + wl < slice_words) {
-        const uint8_t* page = lut_smem + pg * kLutPageBytes;
-        float t[4];
+  for (int pg = 0; pg < NP; ++pg) {
+    const uint8_t* page = lut_smem + pg * kLutPageBytes;
+    const bool live = pg * 16 + wl < slice_words;
+    float t[16][4];
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-          t[s] = *reinterpret_cast<const float*>(page + __byte_perm(wv[p][pg], colb[s], sel[s]));
-        a += (t[0] + t[1]) + (t[2] + t[3]);  // short dependency chains
-      }
-    }
-    acc[p] = a;
+    for (int p = 0; p < 16; ++p)
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        t[p][s] = *reinterpret_cast<const float*>(page + __byte_perm(wv[p][pg], colb[s], sel[s]));
+#pragma unroll
+    for (int p = 0; p < 16; ++p)
+      if (live) acc[p] += (t[p][0] + t[p][1]) + (t[p][2] + t[p][3]);
   }
 
   // ---- 4. reduce-scatter over the 16 lanes of each half: lane wl ends with row pair wl ----
