@@ -44,6 +44,9 @@ class Oracle:
             "oracle_w1a8_acc_at": [_p, _p, _i64, _p, _p, _i64, _p],
             "oracle_w1a8_rescale": [_p, _p, _dbl, _i64, _i64, _p],
             "oracle_w1a1": [_p, _p, _i64, _i64, _i64, _p],
+            "oracle_pack_ternary": [_p, _i64, _i64, _dbl, _p, _p],
+            "oracle_w158a8_acc": [_p, _p, _i64, _i64, _i64, _p],
+            "oracle_w158a8_acc_at": [_p, _p, _i64, _p, _p, _i64, _p],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -143,6 +146,47 @@ class Oracle:
         """Whole BitLinear forward: returns (y fp64, xq, gamma, acc)."""
         xq, gamma = self.ln_absmax_quant(x_bf16, eps)
         acc = self.w1a8_acc(xq, packed, K)
+        return self.w1a8_rescale(acc, gamma, beta), xq, gamma, acc
+
+    # -- b1.58 ternary weights -------------------------------------------------
+    @staticmethod
+    def ternary_row_words(K: int) -> int:
+        return ((K + 127) // 128) * 8
+
+    def pack_ternary(self, W: np.ndarray, eps: float = 1e-5):
+        """b1.58: RoundClip(W / (gamma + eps), -1, 1) as two bit planes per
+        128-k block; returns (packed, gamma = mean |W| in fp64)."""
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        N, K = W.shape
+        packed = np.zeros((N, self.ternary_row_words(K)), dtype=np.uint32)
+        g = np.zeros(1, dtype=np.float64)
+        self._lib.oracle_pack_ternary(_ptr(W), N, K, float(eps), _ptr(packed), _ptr(g))
+        return packed, float(g[0])
+
+    def w158a8_acc(self, xq: np.ndarray, packed: np.ndarray, K: int):
+        xq = np.ascontiguousarray(xq, dtype=np.int8)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        M, N = xq.shape[0], packed.shape[0]
+        assert packed.shape[1] == self.ternary_row_words(K)
+        acc = np.zeros((M, N), dtype=np.int64)
+        self._lib.oracle_w158a8_acc(_ptr(xq), _ptr(packed), M, N, K, _ptr(acc))
+        return acc
+
+    def w158a8_acc_at(self, xq, packed, K: int, ms, js):
+        xq = np.ascontiguousarray(xq, dtype=np.int8)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        ms = np.ascontiguousarray(ms, dtype=np.int64)
+        js = np.ascontiguousarray(js, dtype=np.int64)
+        assert ms.shape == js.shape
+        acc = np.zeros(ms.shape, dtype=np.int64)
+        self._lib.oracle_w158a8_acc_at(_ptr(xq), _ptr(packed), K, _ptr(ms), _ptr(js), ms.size,
+                                       _ptr(acc))
+        return acc
+
+    def w158a8(self, x_bf16, packed, beta: float, K: int, eps: float = 1e-5):
+        """Whole b1.58 BitLinear forward: returns (y fp64, xq, gamma, acc)."""
+        xq, gamma = self.ln_absmax_quant(x_bf16, eps)
+        acc = self.w158a8_acc(xq, packed, K)
         return self.w1a8_rescale(acc, gamma, beta), xq, gamma, acc
 
     # -- W1A1 -----------------------------------------------------------------

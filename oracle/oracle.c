@@ -42,6 +42,19 @@
  *       element (j,k) is bit (k mod 32) of word [j*ceil(K/32) + k/32]; a set
  *       bit means +1, a clear bit -1; unused bits of a row's last word are 0.
  *   R9  Activations are bf16 (raw 16-bit patterns in, decoded exactly).
+ *   R10 b1.58 weights ([BitNet] section 2, Eq.(9)-(11)): the epsilon of
+ *       Eq.(9) is not given; it is a parameter (the library uses 1e-5).
+ *   R11 "round" in Eq.(10): to nearest, ties to even (as R5), applied to
+ *       W / (gamma + eps) evaluated in fp64.
+ *   R12 Packed ternary layout (the library's written spec): row j takes
+ *       ceil(K/128) blocks of 8 uint32 words; block b covers k in
+ *       [128b, 128b + 128): its words 0-3 are the +1 plane, words 4-7 the
+ *       -1 plane, element k at bit (k mod 32) of word (k mod 128)/32 of each
+ *       plane. A weight is +1, -1 or 0 (neither bit set); never both.
+ *   R13 The b1.58 forward is the BitLinear forward of Eq.(7) with the
+ *       ternary weights: the same LN and activation quantisation (section 2
+ *       keeps BitNet's), and the rescale uses gamma of Eq.(11) as beta (Eq.(11)
+ *       and the beta of Eq.(8) are the same mean of |W|).
  */
 #include <math.h>
 #include <stdint.h>
@@ -237,6 +250,71 @@ void oracle_w1a8_rescale(const int64_t* acc, const double* gamma, double beta,
     for (int64_t m = 0; m < M; ++m)
         for (int64_t j = 0; j < N; ++j)
             y[m * N + j] = (double)acc[m * N + j] * beta * gamma[m] / Qb;
+}
+
+/* ---- b1.58 ternary weights ---------------------------------------------- */
+
+static int64_t ternary_row_words(int64_t K) { return ((K + 127) / 128) * 8; }
+
+/* read element (j,k) of a packed ternary matrix as +1 / 0 / -1 (layout R12) */
+static int ternary_value(const uint32_t* packed, int64_t K, int64_t j, int64_t k)
+{
+    const uint32_t* blk = packed + j * ternary_row_words(K) + (k / 128) * 8;
+    int64_t o = k % 128;
+    uint32_t plus = (blk[o / 32] >> (o % 32)) & 1u;
+    uint32_t minus = (blk[4 + o / 32] >> (o % 32)) & 1u;
+    return (int)plus - (int)minus;
+}
+
+/* [BitNet] section 2, Eq.(9)-(11), readings R10-R12:
+ *   gamma  = (1/(N K)) * sum_jk |W_jk|                      (fp64)
+ *   W~_jk  = RoundClip(W_jk / (gamma + eps), -1, 1)
+ *          = max(-1, min(1, round_half_even(W_jk / (gamma + eps))))  */
+void oracle_pack_ternary(const float* W, int64_t N, int64_t K, double eps, uint32_t* packed,
+                         double* gamma_out)
+{
+    double abs_sum = 0.0;
+    for (int64_t j = 0; j < N; ++j)
+        for (int64_t k = 0; k < K; ++k) abs_sum += fabs((double)W[j * K + k]);
+    double gamma = abs_sum / ((double)N * (double)K);
+    memset(packed, 0, (size_t)(N * ternary_row_words(K)) * sizeof(uint32_t));
+    for (int64_t j = 0; j < N; ++j)
+        for (int64_t k = 0; k < K; ++k) {
+            double r = nearbyint((double)W[j * K + k] / (gamma + eps));
+            if (r > 1.0) r = 1.0;
+            if (r < -1.0) r = -1.0;
+            if (r == 0.0) continue;
+            uint32_t* blk = packed + j * ternary_row_words(K) + (k / 128) * 8;
+            int64_t o = k % 128;
+            blk[(r > 0.0 ? 0 : 4) + o / 32] |= 1u << (o % 32);
+        }
+    *gamma_out = gamma;
+}
+
+/* integer core of Eq.(7) with ternary weights (R13):
+ *   acc_mj = sum_k W~_jk * q_mk          (int64) */
+static int64_t w158a8_acc_one(const int8_t* xq, const uint32_t* packed, int64_t K,
+                              int64_t m, int64_t j)
+{
+    int64_t acc = 0;
+    for (int64_t k = 0; k < K; ++k)
+        acc += (int64_t)ternary_value(packed, K, j, k) * (int64_t)xq[m * K + k];
+    return acc;
+}
+
+void oracle_w158a8_acc(const int8_t* xq, const uint32_t* packed, int64_t M, int64_t N,
+                       int64_t K, int64_t* acc)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < N; ++j)
+            acc[m * N + j] = w158a8_acc_one(xq, packed, K, m, j);
+}
+
+void oracle_w158a8_acc_at(const int8_t* xq, const uint32_t* packed, int64_t K,
+                          const int64_t* ms, const int64_t* js, int64_t count, int64_t* acc)
+{
+    for (int64_t i = 0; i < count; ++i)
+        acc[i] = w158a8_acc_one(xq, packed, K, ms[i], js[i]);
 }
 
 /* ---- W1A1 (only as an identity check of the packed-sign reading) ------- */

@@ -17,7 +17,10 @@ What pins what:
 * independent library routines: ``numpy.packbits`` for the packed layout,
   ``math.fsum`` (exact sums) for the scales;
 * invariants: negation, scaling by powers of two, integer shifts, constant
-  tokens, exact .5 ties (round half to even).
+  tokens, exact .5 ties (round half to even);
+* for the b1.58 ternary weights: a hand-worked example with exact ties and
+  clips, equal-magnitude weights reducing to the binary signs (through the
+  separate FBI packing), popcount closed forms, inert sub-threshold weights.
 """
 from __future__ import annotations
 
@@ -310,6 +313,89 @@ def pin_sampled_equals_full(o):
     xq, _ = o.ln_absmax_quant(x)
     acc = o.w1a8_acc(xq, packed, 64)
     assert np.array_equal(o.w1a8_acc_at(xq, packed, 64, ms, js), acc[ms, js])
+
+
+# ---- b1.58 ternary weights (BitNet b1.58 page, section 2, Eq.(9)-(11)) ----
+
+def pin_ternary_example_c_pack(o):
+    ex = _load("ternary_example_c.json")
+    W = np.array([[float(_frac(v)) for v in row] for row in ex["W"]], dtype=np.float32)
+    packed, gamma = o.pack_ternary(W, eps=ex["weight_eps"])
+    assert Fraction(gamma) == _frac(ex["gamma"]), gamma
+    assert packed[:, 0].tolist() == ex["plus_words"], packed
+    assert packed[:, 4].tolist() == ex["minus_words"], packed
+    assert not packed[:, [1, 2, 3, 5, 6, 7]].any(), packed
+
+
+def pin_ternary_example_c_forward(o):
+    ex = _load("ternary_example_c.json")
+    W = np.array([[float(_frac(v)) for v in row] for row in ex["W"]], dtype=np.float32)
+    packed, gamma_w = o.pack_ternary(W, eps=ex["weight_eps"])
+    for tok in ex["tokens"]:
+        x = _bf16_bits_of([_frac(v) for v in tok["x"]])[None, :]
+        xq, gamma = o.ln_absmax_quant(x, ex["ln_eps"])
+        assert xq[0].tolist() == tok["xq"], xq
+        acc = o.w158a8_acc(xq, packed, ex["K"])
+        assert acc[0].tolist() == tok["acc"], acc
+        y = o.w1a8_rescale(acc, gamma, gamma_w)
+        for got, want in zip(y[0], tok["y"]):
+            assert abs(got - float(want)) <= 1e-15 * abs(float(want)), (y, tok["y"])
+
+
+def pin_ternary_equal_magnitudes_are_signs(o):
+    # |W_jk| = c everywhere: gamma = c, W/gamma = +-1, so the ternary weights
+    # are Sign(W) and the b1.58 product equals the binary one (FBI packing)
+    rng = np.random.default_rng(11)
+    N, K = 5, 300
+    W = np.where(rng.random((N, K)) < 0.5, -0.375, 0.375).astype(np.float32)
+    packed_t, gamma = o.pack_ternary(W, eps=0.0)
+    assert gamma == 0.375
+    packed_s, _ = o.pack_fbi(W)
+    xq = rng.integers(-127, 128, size=(3, K), dtype=np.int64).astype(np.int8)
+    assert np.array_equal(o.w158a8_acc(xq, packed_t, K), o.w1a8_acc(xq, packed_s, K))
+
+
+def pin_ternary_all_ones_codes(o):
+    # codes all 1: acc_j = (number of +1 weights) - (number of -1 weights)
+    rng = np.random.default_rng(12)
+    N, K = 7, 260
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    packed, _ = o.pack_ternary(W)
+    xq = np.ones((1, K), dtype=np.int8)
+    acc = o.w158a8_acc(xq, packed, K)[0]
+    w = packed.reshape(N, -1, 8)
+    plus = _popcounts(w[:, :, :4].reshape(N, -1))
+    minus = _popcounts(w[:, :, 4:].reshape(N, -1))
+    assert not (w[:, :, :4] & w[:, :, 4:]).any(), "a weight is both +1 and -1"
+    assert np.array_equal(acc, plus - minus), (acc, plus - minus)
+
+
+def pin_ternary_small_weights_are_inert(o):
+    # weights below half of gamma quantise to 0: changing the codes at those
+    # positions leaves every accumulator unchanged
+    N, K = 3, 128
+    W = np.zeros((N, K), dtype=np.float32)
+    W[:, ::2] = 1.0     # large: ratio 1/gamma > 1/2
+    W[:, 1::2] = 0.125  # small: ratio 0.125/gamma < 1/2
+    packed, gamma = o.pack_ternary(W, eps=0.0)
+    assert gamma == (1.0 + 0.125) / 2
+    rng = np.random.default_rng(13)
+    xq = rng.integers(-127, 128, size=(2, K), dtype=np.int64).astype(np.int8)
+    xq2 = xq.copy()
+    xq2[:, 1::2] = -xq2[:, 1::2] // 2
+    assert np.array_equal(o.w158a8_acc(xq, packed, K), o.w158a8_acc(xq2, packed, K))
+    assert np.array_equal(o.w158a8_acc(xq, packed, K)[:, 0], xq[:, ::2].astype(np.int64).sum(axis=1))
+
+
+def pin_ternary_eps_moves_the_threshold(o):
+    # gamma = 1. eps = 0: every ratio (3/4, 5/4, 1, 1) rounds to 1. eps = 1:
+    # 3/8 rounds to 0, 5/8 to 1, and 1/2 ties to the even 0
+    W = np.array([[0.75, 1.25, 1.0, 1.0]], dtype=np.float32)
+    p0, g0 = o.pack_ternary(W, eps=0.0)
+    p1, g1 = o.pack_ternary(W, eps=1.0)
+    assert g0 == g1 == 1.0
+    assert p0[0, 0] == 0b1111 and p1[0, 0] == 0b0010, (p0, p1)
+    assert p0[0, 4] == 0 and p1[0, 4] == 0
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

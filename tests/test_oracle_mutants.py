@@ -51,6 +51,22 @@ MUTANTS = [
     ("w1a1_and_not_xnor", "s += (int64_t)packed_sign(a, K, m, k) * (int64_t)packed_sign(b, K, j, k);",
      "s += (packed_sign(a, K, m, k) == 1 && packed_sign(b, K, j, k) == 1) ? 1 : -1;"),
     ("bf16_decode_wrong_half", "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+    # b1.58 ternary weights
+    ("ternary_round_half_away", "double r = nearbyint((double)W[j * K + k] / (gamma + eps));",
+     "double r = round((double)W[j * K + k] / (gamma + eps));"),
+    # (dropping the clip altogether is not observable: a +-2 sets the same plane
+    # bit as +-1, so the two-plane layout itself clips)
+    ("ternary_clip_low_to_zero", "if (r < -1.0) r = -1.0;\n            if (r == 0.0) continue;",
+     "if (r < -1.0) r = 0.0;\n            if (r == 0.0) continue;"),
+    ("ternary_gamma_signed_mean", "for (int64_t k = 0; k < K; ++k) abs_sum += fabs((double)W[j * K + k]);",
+     "for (int64_t k = 0; k < K; ++k) abs_sum += (double)W[j * K + k];"),
+    ("ternary_eps_ignored", "/ (gamma + eps));", "/ gamma);"),
+    ("ternary_planes_swapped", "blk[(r > 0.0 ? 0 : 4) + o / 32]", "blk[(r > 0.0 ? 4 : 0) + o / 32]"),
+    ("ternary_block_stride", "(k / 128) * 8;\n    int64_t o = k % 128;\n    uint32_t plus",
+     "(k / 128) * 4;\n    int64_t o = k % 128;\n    uint32_t plus"),
+    ("ternary_acc_sign_ignored",
+     "acc += (int64_t)ternary_value(packed, K, j, k) * (int64_t)xq[m * K + k];",
+     "acc += (int64_t)(ternary_value(packed, K, j, k) != 0) * (int64_t)xq[m * K + k];"),
 ]
 
 
