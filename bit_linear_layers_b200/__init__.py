@@ -9,6 +9,7 @@ if the library is missing, importing the binding raises.
     bin_pack(W, mode)                      -> packed, alpha[, beta]
     bin_linear_w1a16(x, packed, alpha)     -> y (bf16)
     bitlinear_w1a8(x, packed, beta)        -> y (fp32)
+    bitlinear_w158a8(x, packed, beta)      -> y (fp32), b1.58 ternary weights
 """
 from __future__ import annotations
 
@@ -33,11 +34,14 @@ BL_FLAG_OVERLAP_PREVIOUS = 1
 
 BL_PACK_FBI = 0
 BL_PACK_BITNET = 1
+BL_PACK_TERNARY = 2
 
 BL_OP_PACK_FBI = 0
 BL_OP_PACK_BITNET = 1
 BL_OP_W1A16 = 2
 BL_OP_W1A8 = 3
+BL_OP_PACK_TERNARY = 4
+BL_OP_W158A8 = 5
 
 # every symbol include/bitlinear.h declares, with its ctypes signature
 _i64 = ctypes.c_int64
@@ -55,6 +59,8 @@ SIGNATURES = {
     "bitlinear_w1a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
     "bl_device_error": ([_p, _int, ctypes.POINTER(_int)], _int),
     "bitlinear_w1a8_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
+    "bitlinear_w158a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
+    "bitlinear_w158a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
 }
 
 
@@ -123,22 +129,26 @@ def bin_pack(W: torch.Tensor, mode: int = BL_PACK_FBI, *, packed=None, alpha=Non
              ws=None):
     """Binarise W [N, K] fp32 into packed signs [N, K/32] int32 (bit patterns)
     and scales. FBI: returns (packed, alpha[N]). BitNet: returns
-    (packed, alpha[1] = mean W, beta[1] = mean |W|)."""
+    (packed, alpha[1] = mean W, beta[1] = mean |W|). Ternary (b1.58): returns
+    (packed [N, K/16] with a +1 and a -1 plane per 128-k block, beta[1] = mean |W|)."""
     N, K = W.shape
     dev = W.device
+    ternary = mode == BL_PACK_TERNARY
     if packed is None:
-        packed = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
-    if alpha is None:
+        packed = torch.empty((N, K // 16 if ternary else K // 32), dtype=torch.int32, device=dev)
+    if alpha is None and not ternary:
         alpha = torch.empty(N if mode == BL_PACK_FBI else 1, dtype=torch.float32, device=dev)
-    if mode == BL_PACK_BITNET and beta is None:
+    if mode != BL_PACK_FBI and beta is None:
         beta = torch.empty(1, dtype=torch.float32, device=dev)
-    op = BL_OP_PACK_BITNET if mode == BL_PACK_BITNET else BL_OP_PACK_FBI
+    op = {BL_PACK_FBI: BL_OP_PACK_FBI, BL_PACK_BITNET: BL_OP_PACK_BITNET}.get(mode, BL_OP_PACK_TERNARY)
     ws, need = _workspace(op, 0, N, K, dev, ws)
     rc = lib.bin_pack(_dev_ptr(W, torch.float32, "W"), N, K, int(mode),
                       _dev_ptr(packed, torch.int32, "packed"), _dev_ptr(alpha, torch.float32, "alpha"),
                       _dev_ptr(beta, torch.float32, "beta"), _dev_ptr(ws, torch.uint8, "ws"),
                       ws.numel() if ws is not None else 0, _stream(dev))
     _check("bin_pack", rc)
+    if ternary:
+        return packed, beta
     return (packed, alpha) if mode == BL_PACK_FBI else (packed, alpha, beta)
 
 
@@ -198,6 +208,45 @@ def bitlinear_w1a8_debug(x, packed, beta, *, xq_in=None, gamma_in=None, ws=None)
         _dev_ptr(xq_in, torch.int8, "xq_in"), _dev_ptr(gamma_in, torch.float64, "gamma_in"),
         _stream(dev))
     _check("bitlinear_w1a8_debug", rc)
+    return y, xq, gamma, acc
+
+
+def bitlinear_w158a8(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, *, out=None, ws=None):
+    """BitNet b1.58 BitLinear forward: bitlinear_w1a8 with ternary weights
+    (packed from bin_pack(..., BL_PACK_TERNARY), [N, K/16])."""
+    M, K = x.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    ws, _ = _workspace(BL_OP_W158A8, M, N, K, x.device, ws)
+    rc = lib.bitlinear_w158a8(_dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
+                              _dev_ptr(beta, torch.float32, "beta"), _dev_ptr(out, torch.float32, "out"),
+                              M, N, K, _dev_ptr(ws, torch.uint8, "ws"), ws.numel() if ws is not None else 0,
+                              _stream(x.device))
+    _check("bitlinear_w158a8", rc)
+    return out
+
+
+def bitlinear_w158a8_debug(x, packed, beta, *, xq_in=None, gamma_in=None, ws=None):
+    """As bitlinear_w158a8, also returning (xq int8 [M,K], gamma fp64 [M],
+    acc int32 [M,N]). With xq_in/gamma_in the LN/quant step is skipped."""
+    M, K = (xq_in.shape if xq_in is not None else x.shape)
+    N = packed.shape[0]
+    dev = packed.device
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    gamma = torch.empty(M, dtype=torch.float64, device=dev)
+    acc = torch.empty((M, N), dtype=torch.int32, device=dev)
+    ws, _ = _workspace(BL_OP_W158A8, M, N, K, dev, ws)
+    rc = lib.bitlinear_w158a8_debug(
+        _dev_ptr(x, torch.bfloat16, "x") if x is not None else None,
+        _dev_ptr(packed, torch.int32, "packed"), _dev_ptr(beta, torch.float32, "beta"),
+        _dev_ptr(y, torch.float32, "y"), M, N, K, _dev_ptr(ws, torch.uint8, "ws"),
+        ws.numel() if ws is not None else 0, _dev_ptr(xq, torch.int8, "xq"),
+        _dev_ptr(gamma, torch.float64, "gamma"), _dev_ptr(acc, torch.int32, "acc"),
+        _dev_ptr(xq_in, torch.int8, "xq_in"), _dev_ptr(gamma_in, torch.float64, "gamma_in"),
+        _stream(dev))
+    _check("bitlinear_w158a8_debug", rc)
     return y, xq, gamma, acc
 
 

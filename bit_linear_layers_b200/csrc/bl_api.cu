@@ -79,7 +79,7 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<1>, 1 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<2>, 2 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
-              set_ts_smem<0>() && set_ts_smem<1>();
+              set_ts_smem<0>() && set_ts_smem<1>() && set_ts_smem<2>();
     if (!ok) cudaGetLastError();
     for (int S : {2, 4, 8}) {
       cudaLaunchConfig_t cfg = {};
@@ -267,8 +267,8 @@ int launch_ts(const void* act, const uint32_t* packed, int64_t M, int64_t N, int
   const int T = (M >= 256 && 2 * big_tiles >= int64_t(num_sms)) ? 256 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
   CUtensorMap tm_x, tm_bits;
   if (!make_map_2d(&tm_x, act, xt, elem, uint64_t(K), uint64_t(M), 128 / elem, uint32_t(T), CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32), uint64_t(N), 4, 128,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      !make_map_2d(&tm_bits, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(K / 32) * TsCfg<KIND, 1, 32, false>::PLANES,
+                   uint64_t(N), 4 * TsCfg<KIND, 1, 32, false>::PLANES, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
     return BL_ERR_CUDA;
   switch (T) {
     case 256:
@@ -283,9 +283,10 @@ int launch_ts(const void* act, const uint32_t* packed, int64_t M, int64_t N, int
 }
 
 // ---- W1A8 shared body -----------------------------------------------------------
+// `ternary`: packed holds b1.58 weights (two planes, K/16 words per row)
 int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
               int64_t N, int64_t K, void* ws, size_t ws_bytes, int8_t* xq_out, double* gamma_out,
-              int32_t* acc_out, const int8_t* xq_in, const double* gamma_in, void* stream) {
+              int32_t* acc_out, const int8_t* xq_in, const double* gamma_in, bool ternary, void* stream) {
   int rc = check_shape(M, N, K);
   if (rc != BL_OK) return rc;
   if (M == 0) return BL_OK;
@@ -319,17 +320,27 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
 
   if (M <= 16) {
     const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
-    if (M <= 4)
-      gemv_w1a8_kernel<4><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
-    else if (M <= 8)
-      gemv_w1a8_kernel<8><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
-    else
-      gemv_w1a8_kernel<16><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+    if (ternary) {
+      if (M <= 4)
+        gemv_w1a8_kernel<4, true><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+      else if (M <= 8)
+        gemv_w1a8_kernel<8, true><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+      else
+        gemv_w1a8_kernel<16, true><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+    } else {
+      if (M <= 4)
+        gemv_w1a8_kernel<4, false><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+      else if (M <= 8)
+        gemv_w1a8_kernel<8, false><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+      else
+        gemv_w1a8_kernel<16, false><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+    }
     return launch_status();
   }
   int sms = 0;
   device_setup(&sms);
-  return launch_ts<1>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s);
+  return ternary ? launch_ts<2>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s)
+                 : launch_ts<1>(codes, packed, M, N, K, nullptr, gam, beta, y, acc_out, sms, s);
 }
 
 }  // namespace
@@ -359,8 +370,10 @@ const char* bl_status_string(int status) {
 size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
   if (M < 0 || N < 0 || K < 0) return 0;
   switch (op) {
-    case BL_OP_PACK_BITNET: return align256(size_t(N) * 2 * sizeof(double)) + 256;
-    case BL_OP_W1A8: return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double));
+    case BL_OP_PACK_BITNET:
+    case BL_OP_PACK_TERNARY: return align256(size_t(N) * 2 * sizeof(double)) + 256;
+    case BL_OP_W1A8:
+    case BL_OP_W158A8: return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double));
     default: return 0;
   }
 }
@@ -369,9 +382,10 @@ int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, f
              float* beta, void* ws, size_t ws_bytes, void* stream) {
   int rc = check_shape(0, N, K);
   if (rc != BL_OK) return rc;
-  if (mode != BL_PACK_FBI && mode != BL_PACK_BITNET) return BL_ERR_INVALID_ARG;
-  if (!W || !packed || !alpha || !aligned16(W) || !aligned16(packed)) return BL_ERR_INVALID_ARG;
-  if (mode == BL_PACK_BITNET &&
+  if (mode != BL_PACK_FBI && mode != BL_PACK_BITNET && mode != BL_PACK_TERNARY) return BL_ERR_INVALID_ARG;
+  if (!W || !packed || !aligned16(W) || !aligned16(packed)) return BL_ERR_INVALID_ARG;
+  if (mode != BL_PACK_TERNARY && !alpha) return BL_ERR_INVALID_ARG;
+  if (mode != BL_PACK_FBI &&
       (!beta || !ws || !aligned16(ws) || ws_bytes < bl_workspace_bytes(BL_OP_PACK_BITNET, 0, N, K)))
     return BL_ERR_INVALID_ARG;
   int sms = 0;
@@ -389,9 +403,13 @@ int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, f
   double* scalars = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(size_t(N) * 2 * sizeof(double)));
   row_sums_kernel<<<grid, kPackThreads, 0, s>>>(W, N, K, sums);
   if ((rc = launch_status()) != BL_OK) return rc;
-  global_scalars_kernel<<<1, kReduceThreads, 0, s>>>(sums, N, K, scalars, alpha, beta);
+  global_scalars_kernel<<<1, kReduceThreads, 0, s>>>(sums, N, K, scalars,
+                                                      mode == BL_PACK_TERNARY ? nullptr : alpha, beta);
   if ((rc = launch_status()) != BL_OK) return rc;
-  pack_rows_kernel<true><<<grid, kPackThreads, 0, s>>>(W, N, K, packed, nullptr, scalars);
+  if (mode == BL_PACK_TERNARY)
+    pack_ternary_rows_kernel<<<grid, kPackThreads, 0, s>>>(W, N, K, packed, scalars);
+  else
+    pack_rows_kernel<true><<<grid, kPackThreads, 0, s>>>(W, N, K, packed, nullptr, scalars);
   return launch_status();
 }
 
@@ -445,7 +463,21 @@ int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* 
 int bitlinear_w1a8(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
                    int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream) {
   return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, nullptr, nullptr, nullptr, nullptr,
-                   nullptr, stream);
+                   nullptr, false, stream);
+}
+
+int bitlinear_w158a8(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
+                     int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream) {
+  return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, nullptr, nullptr, nullptr, nullptr,
+                   nullptr, true, stream);
+}
+
+int bitlinear_w158a8_debug(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                           int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes, int8_t* xq_out,
+                           double* gamma_out, int32_t* acc_out, const int8_t* xq_in,
+                           const double* gamma_in, void* stream) {
+  return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, xq_out, gamma_out, acc_out, xq_in,
+                   gamma_in, true, stream);
 }
 
 int bitlinear_w1a8_debug(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
@@ -453,7 +485,7 @@ int bitlinear_w1a8_debug(const uint16_t* x, const uint32_t* packed, const float*
                          double* gamma_out, int32_t* acc_out, const int8_t* xq_in,
                          const double* gamma_in, void* stream) {
   return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, xq_out, gamma_out, acc_out, xq_in,
-                   gamma_in, stream);
+                   gamma_in, false, stream);
 }
 
 int bl_device_error(void* stream, int clear, int* where_out) {
@@ -528,5 +560,5 @@ extern "C" int bitlinear_w1a8_noalloc(const uint16_t* x, const uint32_t* packed,
   rc = noalloc_scratch(&scratch);
   if (rc != BL_OK) return rc;
   return w1a8_impl(x, packed, beta, y, M, N, K, scratch, BL_W1A8_NOALLOC_SCRATCH_BYTES, nullptr,
-                   nullptr, nullptr, nullptr, nullptr, stream);
+                   nullptr, nullptr, nullptr, nullptr, false, stream);
 }

@@ -6,6 +6,9 @@
 //   W1A8 ("BitNet b1.58" page, section 1, Eq.(7)-(8)):
 //     acc[m][j] = sum_k s_jk q[m][k]  (exact int32)            kind::i8
 //     y[m][j]   = fp32( acc * beta * gamma_m / 128 )           per-token scale in fp64
+//   W1.58A8 (same page, section 2, Eq.(9)-(11)): as W1A8 with ternary weights
+//     W~_jk in {-1, 0, +1}, stored as a +1 and a -1 bit plane per 128-k block
+//     (KIND 2)
 //
 // The product is computed transposed, D[j][m] = sum_k S[j][k] X[m][k]: the
 // 1-bit weights are the MMA's M side (NB blocks of 128 rows per tile), the
@@ -50,17 +53,20 @@ constexpr int kTsThreads = 512;
 constexpr int kTsExpanders = 8;  // warps
 constexpr int kTsStageK = 128;   // K elements per pipeline stage
 
+// KIND 0: bf16 activations, +-1 weights; 1: int8 codes, +-1 weights;
+// 2: int8 codes, ternary weights (two bit planes per 128-k stage)
 template <int KIND, int NB, int T, bool SPLIT>
 struct TsCfg {
   static constexpr int ROWS = 128 * NB;                         // weight rows per tile
   static constexpr int ELEM = KIND == 0 ? 2 : 1;                // activation bytes
+  static constexpr int PLANES = KIND == 2 ? 2 : 1;              // sign bit planes per weight
   // pipeline unit: one 128-k sign stage; its activations are ATOMS 128-byte
   // swizzle atoms of every token row (64 k each for bf16, 128 k for int8)
   static constexpr int ATOM_K = 128 / ELEM;
   static constexpr int ATOMS = kTsStageK / ATOM_K;              // 2 (bf16) or 1 (int8)
   static constexpr int ATOM_BYTES = T * 128;
   static constexpr int X_UNIT_BYTES = ATOMS * ATOM_BYTES;
-  static constexpr int BITS_BYTES = ROWS * 16;                  // one 128-k sign stage
+  static constexpr int BITS_BYTES = ROWS * 16 * PLANES;         // one 128-k sign stage
   static constexpr int SB = 4;                                  // sign stages in shared memory
   static constexpr int OUT_ELEM = KIND == 0 ? 2 : 4;            // y element bytes
   // the output tile is staged in shared memory and written by bulk tensor
@@ -215,6 +221,17 @@ __device__ __forceinline__ float w1a8_output(int32_t acc, TokScale s) {
   return w1a8_fast_ok(acc) ? w1a8_output_fast(acc, s) : w1a8_output_wide(acc, s);
 }
 
+// 16 ternary weights (16 bits of the +1 plane, 16 of the -1 plane) -> 16
+// int8 values +1 / 0 / -1 in 4 words
+__device__ __forceinline__ void expand16_ternary(uint32_t plus, uint32_t minus, uint32_t* out) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t p = (((plus >> (4 * i)) & 0xFu) * 0x00204081u) & 0x01010101u;
+    const uint32_t m = (((minus >> (4 * i)) & 0xFu) * 0x00204081u) & 0x01010101u;
+    out[i] = p | (m * 0xFFu);
+  }
+}
+
 __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, const uint32_t* v, uint32_t remote_bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
                    remote_addr),
@@ -250,7 +267,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
   __shared__ __align__(8) uint64_t inbox_bar;
   // epilogue scales staged once per tile: beta * gamma / 128 of the tile's tokens (W1A8),
   // alpha of the rows a split-K owner finishes (W1A16)
-  __shared__ TokScale tok_scale[KIND == 1 ? T : 1];
+  __shared__ TokScale tok_scale[KIND != 0 ? T : 1];
   __shared__ float row_alpha[SPLIT && KIND == 0 ? ROWS : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -319,7 +336,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
           }
           const uint32_t bb = smem_u32(&b_full[bs]);
           mbar_arrive_expect_tx(bb, C::BITS_BYTES);
-          tma_load_2d(smem_u32(bits_ring + bs * C::BITS_BYTES), &tm_bits, bb, u * 4, w0);
+          tma_load_2d(smem_u32(bits_ring + bs * C::BITS_BYTES), &tm_bits, bb, u * 4 * C::PLANES, w0);
           const uint32_t xs = it % SX;
           if (it >= SX && !mbar_wait(smem_u32(&x_empty[xs]), ((it / SX) - 1) & 1, kWhereGemmProducer)) {
             ok = false;
@@ -413,8 +430,11 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     auto expand_and_store = [&](uint32_t it) {
       tc_fence_after_sync();
       const uint32_t a = it % SA, bs = it % C::SB;
-      const uint4 wv = *reinterpret_cast<const uint4*>(bits_ring + bs * C::BITS_BYTES + r * 16);
+      const uint4 wv = *reinterpret_cast<const uint4*>(bits_ring + bs * C::BITS_BYTES + r * 16 * C::PLANES);
       const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+      uint4 mv = make_uint4(0u, 0u, 0u, 0u);
+      if (KIND == 2) mv = *reinterpret_cast<const uint4*>(bits_ring + bs * C::BITS_BYTES + r * 32 + 16);
+      const uint32_t md[4] = {mv.x, mv.y, mv.z, mv.w};
       const uint32_t taddr = a_base + (a * NB + blk) * C::A_COLS + ch0 * COLS_PER_CH +
                              (static_cast<uint32_t>(q * 32) << 16);
       // this warp's chunks are words ch0/2 .. ch0/2 + MY_CH/2 - 1 of the row
@@ -422,10 +442,14 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
       for (int j = 0; j < MY_CH; ++j) {
         const uint32_t word = NB == 2 ? wd[j >> 1] : (ch0 == 0 ? wd[j >> 1] : wd[2 + (j >> 1)]);
         const uint32_t chunk = (word >> (16 * (j & 1))) & 0xFFFFu;  // ch0 is even
-        if (KIND == 0)
+        if (KIND == 0) {
           expand16_bf16(chunk, v + j * COLS_PER_CH);
-        else
+        } else if (KIND == 1) {
           expand16_i8(chunk, v + j * COLS_PER_CH);
+        } else {
+          const uint32_t mword = NB == 2 ? md[j >> 1] : (ch0 == 0 ? md[j >> 1] : md[2 + (j >> 1)]);
+          expand16_ternary(chunk, (mword >> (16 * (j & 1))) & 0xFFFFu, v + j * COLS_PER_CH);
+        }
       }
       tmem_st_wide<MY_CH * COLS_PER_CH>(taddr, v);
     };
@@ -458,7 +482,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     const int tile = tile_first;
     const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
     // scales of the rows this CTA finishes / of the tile's tokens, read while the MMAs run
-    if (KIND == 1) {
+    if (KIND != 0) {
       const double bt = static_cast<double>(*beta);
       for (int tt = et; tt < T; tt += 128)
         tok_scale[tt] = w1a8_token_scale(bt, t0 + tt < M ? gamma[t0 + tt] : 0.0);
@@ -545,10 +569,10 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     const bool leader = (warp == 4 && lane == 0);
     uint32_t tcount = 0;
     double bt = 0.0;
-    if (KIND == 1) bt = static_cast<double>(*beta);
+    if (KIND != 0) bt = static_cast<double>(*beta);
     for (int tile = tile_first; tile < num_tiles; tile += tile_step, ++tcount) {
       const int t0 = (tile % tiles_t) * T, w0 = (tile / tiles_t) * ROWS;
-      if (KIND == 1) {
+      if (KIND != 0) {
         epilogue_bar();  // the previous tile's readers of tok_scale are done
         for (int tt = et; tt < T; tt += 128)
           tok_scale[tt] = w1a8_token_scale(bt, t0 + tt < M ? gamma[t0 + tt] : 0.0);

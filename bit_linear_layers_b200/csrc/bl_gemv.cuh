@@ -117,14 +117,24 @@ __device__ __forceinline__ uint32_t nibble_to_pm1_i8(uint32_t nib) {
   return spread * 0xFFFFFF02u + 0xFFFFFFFFu;                  // 1 -> 0x01, 0 -> 0xFF
 }
 
-template <int MT>
+// four ternary weights (a +1 nibble and a -1 nibble) -> four int8 lanes of +1 / 0 / -1
+__device__ __forceinline__ uint32_t nibbles_to_ternary_i8(uint32_t plus, uint32_t minus) {
+  const uint32_t p = (plus * 0x00204081u) & 0x01010101u;   // bit i -> byte i = 1
+  const uint32_t m = (minus * 0x00204081u) & 0x01010101u;
+  return p | (m * 0xFFu);                                   // -1 bytes: 0xFF (never both)
+}
+
+// kTernary: `packed` holds b1.58 weights, per 128-k block 4 words of the +1
+// plane then 4 of the -1 plane (row stride K/16 words)
+template <int MT, bool kTernary>
 __global__ void __launch_bounds__(kGemvThreads) gemv_w1a8_kernel(
     const int8_t* __restrict__ xq, const double* __restrict__ gamma,
     const uint32_t* __restrict__ packed, const float* __restrict__ beta, float* __restrict__ y,
     int32_t* __restrict__ acc_out, int M, int64_t N, int64_t K) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kGemvRowsPerCta + warp * kGemvRowsPerWarp;
-  const int64_t words = K / 32;
+  const int64_t words = K / 32;  // 32-k groups per row
+  const int64_t stride = kTernary ? K / 16 : K / 32;
   int acc[kGemvRowsPerWarp][MT];
 #pragma unroll
   for (int r = 0; r < kGemvRowsPerWarp; ++r)
@@ -132,11 +142,13 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_w1a8_kernel(
     for (int m = 0; m < MT; ++m) acc[r][m] = 0;
 
   for (int64_t wi = lane; wi < words; wi += 32) {
-    uint32_t wr[kGemvRowsPerWarp];
+    uint32_t wr[kGemvRowsPerWarp], wm[kGemvRowsPerWarp];
+    const int64_t off = kTernary ? (wi >> 2) * 8 + (wi & 3) : wi;
 #pragma unroll
     for (int r = 0; r < kGemvRowsPerWarp; ++r) {
       const int64_t row = row0 + r;
-      wr[r] = row < N ? __ldcs(packed + row * words + wi) : 0u;
+      wr[r] = row < N ? __ldcs(packed + row * stride + off) : 0u;
+      wm[r] = (kTernary && row < N) ? __ldcs(packed + row * stride + off + 4) : 0u;
     }
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
@@ -148,9 +160,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_w1a8_kernel(
       for (int r = 0; r < kGemvRowsPerWarp; ++r) {
         int a = acc[r][m];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          a = __dp4a(static_cast<int>(nibble_to_pm1_i8((wr[r] >> (4 * i)) & 0xFu)),
-                     static_cast<int>(xv[i]), a);
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t wbytes = kTernary
+                                      ? nibbles_to_ternary_i8((wr[r] >> (4 * i)) & 0xFu, (wm[r] >> (4 * i)) & 0xFu)
+                                      : nibble_to_pm1_i8((wr[r] >> (4 * i)) & 0xFu);
+          a = __dp4a(static_cast<int>(wbytes), static_cast<int>(xv[i]), a);
+        }
         acc[r][m] = a;
       }
     }

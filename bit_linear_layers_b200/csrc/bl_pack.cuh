@@ -3,7 +3,9 @@
 // FBI-linear ("FBI-LLM" page, FBI-linear paragraph): bit = W > 0 and one
 // scale per output channel, alpha_j = mean_k |W_jk| (fp64 sum, one rounding
 // to fp32). BitNet ("BitNet b1.58" page, section 1, Eq.(1)-(3), (8)):
-// bit = (W - mean W) > 0 compared in fp64, beta = mean |W|.
+// bit = (W - mean W) > 0 compared in fp64, beta = mean |W|. b1.58 ("BitNet
+// b1.58" page, section 2, Eq.(9)-(11)): W~ = RoundClip(W / (gamma + eps), -1, 1)
+// with gamma = mean |W|, as a +1 and a -1 bit plane per 128-k block.
 //
 // A warp owns one row at a time and sweeps it 128 floats per step: each lane
 // loads a float4, turns it into a 4-bit nibble, and an OR-reduction over each
@@ -85,6 +87,42 @@ __global__ void __launch_bounds__(kPackThreads) pack_rows_kernel(
     if (!kBitNet) {
       abs_sum = warp_sum(abs_sum);
       if (lane == 0) alpha[row] = static_cast<float>(abs_sum / static_cast<double>(K));
+    }
+  }
+}
+
+// b1.58 ternary pass (after row_sums_kernel and global_scalars_kernel, whose
+// scalars[1] is gamma = mean |W| in fp64). q = W / (gamma + eps) is divided in
+// fp64 exactly as the formula reads; round-half-even then clip to [-1, 1] is
+// +1 for q > 1/2, -1 for q < -1/2 and 0 otherwise (q = +-1/2 ties to 0).
+// Row layout: per 128-k block, 4 words of the +1 plane then 4 of the -1 plane.
+constexpr double kTernaryEps = 1e-5;
+__global__ void __launch_bounds__(kPackThreads) pack_ternary_rows_kernel(
+    const float* __restrict__ W, int64_t N, int64_t K, uint32_t* __restrict__ packed,
+    const double* __restrict__ scalars) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const double d = scalars[1] + kTernaryEps;
+  const int64_t steps = K / 128;  // one 128-k block per warp step
+  for (int64_t row = warp0; row < N; row += nwarps) {
+    const float4* src = reinterpret_cast<const float4*>(W + row * K) + lane;
+    uint32_t* dst = packed + row * (K / 16) + (lane >> 3);
+    for (int64_t s = 0; s < steps; ++s) {
+      const float4 v = __ldcs(src + s * 32);
+      const double q[4] = {static_cast<double>(v.x) / d, static_cast<double>(v.y) / d,
+                           static_cast<double>(v.z) / d, static_cast<double>(v.w) / d};
+      uint32_t plus = 0u, minus = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        plus |= (q[i] > 0.5 ? 1u : 0u) << i;
+        minus |= (q[i] < -0.5 ? 1u : 0u) << i;
+      }
+      const uint32_t pw = nibble_words(plus, lane), mw = nibble_words(minus, lane);
+      if ((lane & 7) == 0) {
+        dst[s * 8] = pw;
+        dst[s * 8 + 4] = mw;
+      }
     }
   }
 }

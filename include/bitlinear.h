@@ -55,14 +55,17 @@ extern "C" {
                                   /* bitlinear_w1a8_noalloc                         */
 
 /* ---- bin_pack modes ----------------------------------------------------- */
-#define BL_PACK_FBI 0    /* sign(W), per-output-channel alpha                 */
-#define BL_PACK_BITNET 1 /* sign(W - mean W), global alpha and beta           */
+#define BL_PACK_FBI 0     /* sign(W), per-output-channel alpha                */
+#define BL_PACK_BITNET 1  /* sign(W - mean W), global alpha and beta          */
+#define BL_PACK_TERNARY 2 /* b1.58: RoundClip(W / (mean|W| + eps)), two planes */
 
 /* ---- ops for bl_workspace_bytes ----------------------------------------- */
 #define BL_OP_PACK_FBI 0
 #define BL_OP_PACK_BITNET 1
 #define BL_OP_W1A16 2
 #define BL_OP_W1A8 3
+#define BL_OP_PACK_TERNARY 4
+#define BL_OP_W158A8 5
 
 /* Library ABI version (this header: 1). */
 int bl_abi_version(void);
@@ -88,7 +91,17 @@ size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
  *   beta = (1/NK) * sum |W| (fp64, unshifted W).
  *   alpha[0] = (float)a (informational), beta[0] = (float)beta.
  *   Needs ws of bl_workspace_bytes(BL_OP_PACK_BITNET, 0, N, K) bytes.
- * Outputs: packed [N x K/32] uint32 (layout above). All device pointers.
+ * mode BL_PACK_TERNARY ("BitNet b1.58" page, section 2, Eq.(9)-(11)):
+ *   g = (1/NK) * sum |W| (fp64);  W~_jk = RoundClip(W_jk / (g + 1e-5), -1, 1)
+ *   with round half to even and the division in fp64 (so +1 iff the quotient
+ *   exceeds 1/2, -1 iff it is below -1/2, else 0). beta[0] = (float)g, the
+ *   scale of the forward; `alpha` is unused (may be NULL). packed is
+ *   [N x K/16] uint32: per row, per 128-k block, 4 words of the +1 plane then
+ *   4 words of the -1 plane (element k at bit k mod 32 of word (k mod 128)/32
+ *   of each plane; never both bits). Needs ws of
+ *   bl_workspace_bytes(BL_OP_PACK_TERNARY, 0, N, K) bytes.
+ * Outputs: packed [N x K/32] uint32 (layout above; [N x K/16] for
+ * BL_PACK_TERNARY). All device pointers.
  */
 int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, float* alpha,
              float* beta, void* ws, size_t ws_bytes, void* stream);
@@ -151,6 +164,25 @@ int bitlinear_w1a8_debug(const uint16_t* x, const uint32_t* packed, const float*
                          int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
                          int8_t* xq_out, double* gamma_out, int32_t* acc_out,
                          const int8_t* xq_in, const double* gamma_in, void* stream);
+
+/*
+ * bitlinear_w158a8 -- BitNet b1.58 BitLinear forward ("BitNet b1.58" page,
+ * section 2: the ternary weights of Eq.(9)-(11) in the forward of section 1,
+ * whose LN and activation quantisation b1.58 keeps). Exactly bitlinear_w1a8
+ * with acc[m][j] = sum_k W~_jk * q_mk (W~ in {-1, 0, +1}, exact int32) and
+ * beta = the mean |W| from bin_pack(BL_PACK_TERNARY). packed [N x K/16]
+ * (two planes, layout of BL_PACK_TERNARY). Needs ws of
+ * bl_workspace_bytes(BL_OP_W158A8, M, N, K) bytes (same as BL_OP_W1A8).
+ */
+int bitlinear_w158a8(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                     int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream);
+
+/* bitlinear_w158a8_debug -- bitlinear_w158a8 with the extra outputs and
+ * inputs of bitlinear_w1a8_debug. */
+int bitlinear_w158a8_debug(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                           int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
+                           int8_t* xq_out, double* gamma_out, int32_t* acc_out,
+                           const int8_t* xq_in, const double* gamma_in, void* stream);
 
 /*
  * bl_device_error -- synchronise `stream`, then return the first in-kernel
