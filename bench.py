@@ -2,7 +2,7 @@
 """Benchmark of the binarized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|w1a8] [--no-secondary]
+                    [--workload decode|prefill|w1a8|w158a8] [--no-secondary]
 
 Workloads (a step is one pass of the layer over one batch of synthetic input):
 
@@ -14,7 +14,8 @@ Workloads (a step is one pass of the layer over one batch of synthetic input):
   TFLOP/s against the measured bf16 tensor peak;
 * ``w1a8``: BitNet BitLinear (LN + absmax int8 quantisation + int8 GEMM +
   rescale) on the 1.3B shapes, 512 tokens, 2048->5632 then 5632->2048, in
-  TOP/s against the int8 tensor peak.
+  TOP/s against the int8 tensor peak;
+* ``w158a8``: the same with BitNet b1.58 ternary weights.
 
 Each workload keeps R distinct copies of its weights and activations whose
 total is more than twice the 126 MB L2, and step i uses copy i % R, so no step
@@ -423,7 +424,74 @@ class W1A8(Workload):
             self.o.w1a8(x, p, beta, K)
 
 
-WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8)}
+class W158A8(W1A8):
+    """BitNet b1.58: the W1A8 workload with ternary weights (RoundClip of
+    W / mean|W|, two bit planes)."""
+    name = "w158a8"
+    metric = "BitLinear b1.58 W1.58A8 TOP/s (1.3B shapes, 512 tokens, ternary weights)"
+    kernel = "ln_quant_kernel + gemm_ts_kernel<2,1,T,*> (one call; time includes LN + quantisation)"
+    traffic_file = None
+
+    def __init__(self):
+        super().__init__()
+        self.config = dict(self.config)
+        self.config["workload"] = ("BitNet b1.58 BitLinear W1.58A8, 512 tokens, 1.3B shapes 2048->5632 then "
+                                   "5632->2048, ternary weights")
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        from bit_linear_layers_b200 import synthetic
+        self.bl = bl
+        self.copies = []
+        for i in range(self.rotate):
+            layers = []
+            for s, (M, K, N) in enumerate(self.SHAPES):
+                seed = 4 + 100 * i + 10 * s + 7 * rank
+                W = synthetic.weights(N, K, seed=seed, mean=0.001, device=dev)
+                p, b = bl.bin_pack(W, bl.BL_PACK_TERNARY)
+                del W
+                x = synthetic.laplace_channel_activations(M, K, seed=seed, device=dev)
+                ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W158A8, M, N, K), dtype=torch.uint8, device=dev)
+                y = torch.empty((M, N), dtype=torch.float32, device=dev)
+                layers.append((x, p, b, ws, y))
+            self.copies.append(layers)
+        self.xh = [lay[0].cpu().pin_memory() for lay in self.copies[0]]
+        self.yh = [torch.empty_like(lay[4], device="cpu").pin_memory() for lay in self.copies[0]]
+        self.h2d = sum(M * K * 2 for M, K, N in self.SHAPES)
+        self.d2h = sum(M * N * 4 for M, K, N in self.SHAPES)
+
+    def step(self, i):
+        for x, p, b, ws, y in self.copies[i % self.rotate]:
+            self.bl.bitlinear_w158a8(x, p, b, out=y, ws=ws)
+
+    def e2e_step(self, i):
+        for (x, p, b, ws, y), xh, yh in zip(self.copies[i % self.rotate], self.xh, self.yh):
+            x.copy_(xh, non_blocking=True)
+            self.bl.bitlinear_w158a8(x, p, b, out=y, ws=ws)
+            yh.copy_(y, non_blocking=True)
+
+    def oracle_setup(self):
+        import oracle as oracle_pkg
+        from bit_linear_layers_b200 import synthetic
+        self.o = oracle_pkg.get()
+        self.olayers, ops = [], 0.0
+        for s, (M, K, N) in enumerate(self.SHAPES):
+            W = synthetic.weights(N, K, seed=4 + 10 * s, mean=0.001).numpy()
+            p, gamma_w = self.o.pack_ternary(W)  # gamma needs the whole matrix
+            x = synthetic.bf16_bits(synthetic.laplace_channel_activations(1, K, seed=4 + 10 * s))
+            self.olayers.append((x, p[:self.ORACLE_COLS].copy(), gamma_w, K))
+            ops += 2.0 * K * self.ORACLE_COLS
+        self.oracle_sample = ("one token through LN + quantisation and output columns 0..1023 of both "
+                              "projections per call, ternary weights (single-threaded C oracle, fp64/int64)")
+        return ops
+
+    def oracle_call(self):
+        for x, p, gamma_w, K in self.olayers:
+            self.o.w158a8(x, p, gamma_w, K)
+
+
+WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8, W158A8)}
 
 
 # ----------------------------------------------------------------------------- ours
