@@ -2,7 +2,7 @@
 """Benchmark of the binarized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|w1a8|w158a8] [--no-secondary]
+                    [--workload decode|prefill|w1a8|w158a8|w1a1] [--no-secondary]
 
 Workloads (a step is one pass of the layer over one batch of synthetic input):
 
@@ -15,7 +15,9 @@ Workloads (a step is one pass of the layer over one batch of synthetic input):
 * ``w1a8``: BitNet BitLinear (LN + absmax int8 quantisation + int8 GEMM +
   rescale) on the 1.3B shapes, 512 tokens, 2048->5632 then 5632->2048, in
   TOP/s against the int8 tensor peak;
-* ``w158a8``: the same with BitNet b1.58 ternary weights.
+* ``w158a8``: the same with BitNet b1.58 ternary weights;
+* ``w1a1``: XNOR/popcount products of packed +-1 operands at the same shapes,
+  against a population-count (integer ALU) roofline.
 
 Each workload keeps R distinct copies of its weights and activations whose
 total is more than twice the 126 MB L2, and step i uses copy i % R, so no step
@@ -491,7 +493,89 @@ class W158A8(W1A8):
             self.o.w158a8(x, p, gamma_w, K)
 
 
-WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8, W158A8)}
+class W1A1(Workload):
+    """W1A1 XNOR/popcount products at the 1.3B shapes, 512 tokens, on packed
+    +-1 activations and weights. Bound by population-count throughput."""
+    name = "w1a1"
+    SHAPES = [(512, 2048, 5632), (512, 5632, 2048)]
+    metric = "W1A1 XNOR-popcount TOP/s (1.3B shapes, 512 tokens, packed +-1 operands)"
+    unit, scale, bound = "TOP/s", 1e12, "alu"
+    dtype = "b1"
+    kernel = "xnor_gemm_kernel (64x64 tiles, XOR + POPC on the integer pipes)"
+    sources = [CSRC + "bl_xnor.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    launches_per_step = 2
+    rotate = 8
+    # 16 population counts per SM per clock (each one 32 +-1 products), 2 ops
+    # per product, at the maximum SM clock
+    POPC_PER_SM_CLK = 16
+
+    def __init__(self):
+        per_copy = sum(M * K // 8 + N * K // 8 + M * N * 4 for M, K, N in self.SHAPES)
+        self.config = {"workload": "W1A1 XNOR-popcount products, 512 tokens, 1.3B shapes 2048->5632 then 5632->2048",
+                       "shapes_MKN": [list(s) for s in self.SHAPES],
+                       "l2": f"{self.rotate} rotating copies ({self.rotate * per_copy / 1e6:.0f} MB); the packed "
+                             "operands are small (L2-resident), the int32 outputs stream"}
+
+    def units_per_step(self):
+        return sum(2.0 * M * K * N for M, K, N in self.SHAPES)
+
+    def peak(self, peaks, timed_s):
+        sms, mhz = 148, 1965.0
+        p = sms * self.POPC_PER_SM_CLK * 32 * 2 * mhz * 1e6 / 1e12
+        return p, f"derived: {sms} SMs x {self.POPC_PER_SM_CLK} popc/clk x 32 products x 2 ops x {mhz:.0f} MHz"
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        self.bl = bl
+        g = torch.Generator(device=dev)
+        g.manual_seed(replica_seed(31, 1, rank))
+        self.copies = []
+        for i in range(self.rotate):
+            layers = []
+            for (M, K, N) in self.SHAPES:
+                a = torch.randint(-2 ** 31, 2 ** 31 - 1, (M, K // 32), generator=g, dtype=torch.int32, device=dev)
+                b = torch.randint(-2 ** 31, 2 ** 31 - 1, (N, K // 32), generator=g, dtype=torch.int32, device=dev)
+                layers.append((a, b, K, torch.empty((M, N), dtype=torch.int32, device=dev)))
+            self.copies.append(layers)
+        self.ah = [lay[0].cpu().pin_memory() for lay in self.copies[0]]
+        self.yh = [torch.empty_like(lay[3], device="cpu").pin_memory() for lay in self.copies[0]]
+        self.h2d = sum(M * K // 8 for M, K, N in self.SHAPES)
+        self.d2h = sum(M * N * 4 for M, K, N in self.SHAPES)
+
+    def step(self, i):
+        for a, b, K, y in self.copies[i % self.rotate]:
+            self.bl.bin_xnor_gemm(a, b, K, out=y)
+
+    def e2e_step(self, i):
+        for (a, b, K, y), ah, yh in zip(self.copies[i % self.rotate], self.ah, self.yh):
+            a.copy_(ah, non_blocking=True)
+            self.bl.bin_xnor_gemm(a, b, K, out=y)
+            yh.copy_(y, non_blocking=True)
+
+    ORACLE_COLS = 256
+
+    def oracle_setup(self):
+        import numpy as np
+        import oracle as oracle_pkg
+        self.o = oracle_pkg.get()
+        rng = np.random.default_rng(31)
+        self.olayers, ops = [], 0.0
+        for (M, K, N) in self.SHAPES:
+            a = rng.integers(0, 2 ** 32, size=(1, K // 32), dtype=np.uint64).astype(np.uint32)
+            b = rng.integers(0, 2 ** 32, size=(self.ORACLE_COLS, K // 32), dtype=np.uint64).astype(np.uint32)
+            self.olayers.append((a, b, K))
+            ops += 2.0 * K * self.ORACLE_COLS
+        self.oracle_sample = ("one packed token against 256 packed rows of both shapes per call "
+                              "(single-threaded C oracle, bit by bit)")
+        return ops
+
+    def oracle_call(self):
+        for a, b, K in self.olayers:
+            self.o.w1a1(a, b, K)
+
+
+WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8, W158A8, W1A1)}
 
 
 # ----------------------------------------------------------------------------- ours

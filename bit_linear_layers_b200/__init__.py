@@ -59,6 +59,7 @@ SIGNATURES = {
     "bitlinear_w1a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
     "bl_device_error": ([_p, _int, ctypes.POINTER(_int)], _int),
     "bitlinear_w1a8_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
+    "bin_xnor_gemm": ([_p, _p, _p, _i64, _i64, _i64, _p], _int),
     "bitlinear_w158a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w158a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
 }
@@ -263,6 +264,18 @@ def bitlinear_w1a8_noalloc(x: torch.Tensor, packed: torch.Tensor, beta: torch.Te
                                     _dev_ptr(beta, torch.float32, "beta"), _dev_ptr(out, torch.float32, "out"),
                                     M, N, K, _stream(x.device))
     _check("bitlinear_w1a8_noalloc", rc)
+    return out
+
+
+def bin_xnor_gemm(a: torch.Tensor, b: torch.Tensor, K: int, *, out=None):
+    """W1A1: dot[m, n] = K - 2 * popcount(a[m] XOR b[n]) for packed +-1 rows
+    a [M, K/32] and b [N, K/32] (int32 bit patterns); returns int32 [M, N]."""
+    M, N = a.shape[0], b.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.int32, device=a.device)
+    rc = lib.bin_xnor_gemm(_dev_ptr(a, torch.int32, "a"), _dev_ptr(b, torch.int32, "b"),
+                           _dev_ptr(out, torch.int32, "out"), M, N, K, _stream(a.device))
+    _check("bin_xnor_gemm", rc)
     return out
 
 

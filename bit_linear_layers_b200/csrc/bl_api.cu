@@ -17,6 +17,7 @@
 #include "bl_gemv_lut.cuh"
 #include "bl_lnquant.cuh"
 #include "bl_pack.cuh"
+#include "bl_xnor.cuh"
 
 namespace bl {
 namespace {
@@ -486,6 +487,21 @@ int bitlinear_w1a8_debug(const uint16_t* x, const uint32_t* packed, const float*
                          const double* gamma_in, void* stream) {
   return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, xq_out, gamma_out, acc_out, xq_in,
                    gamma_in, false, stream);
+}
+
+int bin_xnor_gemm(const uint32_t* a, const uint32_t* b, int32_t* dot, int64_t M, int64_t N, int64_t K,
+                  void* stream) {
+  int rc = check_shape(M, N, K);
+  if (rc != BL_OK) return rc;
+  if (M == 0) return BL_OK;
+  if (K > (int64_t(1) << 30)) return BL_ERR_UNSUPPORTED;  // dot must fit int32
+  if (!a || !b || !dot) return BL_ERR_INVALID_ARG;
+  rc = device_setup(nullptr);
+  if (rc != BL_OK) return rc;
+  if (cdiv(M, kXnorTile) > 65535) return BL_ERR_UNSUPPORTED;  // grid y limit
+  const dim3 grid(static_cast<unsigned>(cdiv(N, kXnorTile)), static_cast<unsigned>(cdiv(M, kXnorTile)), 1);
+  xnor_gemm_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a, b, dot, M, N, K);
+  return launch_status();
 }
 
 int bl_device_error(void* stream, int clear, int* where_out) {

@@ -185,6 +185,17 @@ int bitlinear_w158a8_debug(const uint16_t* x, const uint32_t* packed, const floa
                            const int8_t* xq_in, const double* gamma_in, void* stream);
 
 /*
+ * bin_xnor_gemm -- W1A1: products of two +-1 matrices ("BitNet-Transformers"
+ * page: 1-bit operands reduce the product to XNOR / popcount arithmetic):
+ *   dot[m][n] = sum_k a_mk * b_nk = K - 2 * popcount(a_m XOR b_n)   (exact int32)
+ * a [M x K/32] and b [N x K/32] uint32 in the packed sign layout (bit set =
+ * +1); e.g. both from bin_pack(..., BL_PACK_FBI), whose alpha output is then
+ * ignored. dot [M x N] int32. Device pointers; K a multiple of 128.
+ */
+int bin_xnor_gemm(const uint32_t* a, const uint32_t* b, int32_t* dot, int64_t M, int64_t N, int64_t K,
+                  void* stream);
+
+/*
  * bl_device_error -- synchronise `stream`, then return the first in-kernel
  * fault recorded on the current device since the last clear (BL_OK if none;
  * BL_ERR_TIMEOUT when a bounded wait ran out). If `clear` is non-zero the
