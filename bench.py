@@ -692,8 +692,8 @@ def summarize(wl, ms, ms_e2e, steps, world, peaks, peak_kind):
     achieved = wl.achieved(per_step_s)
     roof = {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": wl.unit,
             "frac": achieved / peak, "traffic": wl.traffic(), "kernel": wl.kernel,
-            "peak_source": f"{peak_kind}: MEASURED_PEAKS.json {peak_key}" if peak_kind == "measured"
-            else f"fallback ({peak_key})"}
+            "peak_source": peak_key if peak_key.startswith("derived")
+            else (f"{peak_kind}: MEASURED_PEAKS.json {peak_key}" if peak_kind == "measured" else f"fallback ({peak_key})")}
     if isinstance(wl, Decode):
         roof["algorithmic_bytes_per_launch"] = wl.alg_b
     value = whole_job_value(world, steps, wl.units_per_step(), ms, wl.scale)
