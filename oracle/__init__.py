@@ -45,6 +45,7 @@ class Oracle:
             "oracle_w1a8_rescale": [_p, _p, _dbl, _i64, _i64, _p],
             "oracle_w1a1": [_p, _p, _i64, _i64, _i64, _p],
             "oracle_pack_ternary": [_p, _i64, _i64, _dbl, _p, _p],
+            "oracle_ln_quant_tensor": [_p, _i64, _i64, _dbl, ctypes.c_int, _p, _p, _p, _p],
             "oracle_w158a8_acc": [_p, _p, _i64, _i64, _i64, _p],
             "oracle_w158a8_acc_at": [_p, _p, _i64, _p, _p, _i64, _p],
         }
@@ -114,6 +115,20 @@ class Oracle:
         self._lib.oracle_ln_absmax_quant(_ptr(x), M, K, float(eps), _ptr(xq), _ptr(gamma),
                                          _ptr(pre) if want_pre else None)
         return (xq, gamma, pre) if want_pre else (xq, gamma)
+
+    def ln_quant_tensor(self, x_bf16: np.ndarray, mode: int, eps: float = 1e-5, want_pre: bool = False):
+        """Per-tensor quantisation of the LN output: mode 0 = Eq.(5) over the
+        whole matrix (codes in [-127, 127]), mode 1 = Eq.(6) (shift by the
+        minimum, codes in [0, 127]). Returns (xq, gamma [M] (all equal), eta[, pre])."""
+        x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+        M, K = x.shape
+        xq = np.zeros((M, K), dtype=np.int8)
+        gamma = np.zeros(M, dtype=np.float64)
+        eta = np.zeros(1, dtype=np.float64)
+        pre = np.zeros((M, K), dtype=np.float64) if want_pre else None
+        self._lib.oracle_ln_quant_tensor(_ptr(x), M, K, float(eps), int(mode), _ptr(xq), _ptr(gamma),
+                                         _ptr(eta), _ptr(pre) if want_pre else None)
+        return (xq, gamma, float(eta[0]), pre) if want_pre else (xq, gamma, float(eta[0]))
 
     def w1a8_acc(self, xq: np.ndarray, packed: np.ndarray, K: int):
         xq = np.ascontiguousarray(xq, dtype=np.int8)

@@ -51,6 +51,15 @@
  *       [128b, 128b + 128): its words 0-3 are the +1 plane, words 4-7 the
  *       -1 plane, element k at bit (k mod 32) of word (k mod 128)/32 of each
  *       plane. A weight is +1, -1 or 0 (neither bit set); never both.
+ *   R14 Per-tensor activation scale ([BitNet] Eq.(5) literally: "of the input
+ *       matrix"): gamma = max |LN(x)| over all M x K elements, shared by all
+ *       tokens; codes as R5.
+ *   R15 Eq.(6) (activations before a nonlinearity): eta = min over all M x K
+ *       LN values, gamma = max over all of (LN - eta), so (LN - eta) * Q_b /
+ *       gamma lies in [0, Q_b]; rounded to nearest (ties to even) and clamped
+ *       to [0, 127] (the clip bounds eps and Q_b - eps as integers). The
+ *       forward then applies Eq.(7) as printed, y = acc * beta * gamma / Q_b
+ *       (the pages give no term for eta). gamma == 0 gives all-zero codes.
  *   R13 The b1.58 forward is the BitLinear forward of Eq.(7) with the
  *       ternary weights: the same LN and activation quantisation (section 2
  *       keeps BitNet's), and the rescale uses gamma of Eq.(11) as beta (Eq.(11)
@@ -214,6 +223,63 @@ void oracle_ln_absmax_quant(const uint16_t* x, int64_t M, int64_t K, double eps,
             xq[m * K + k] = (int8_t)r;
         }
     }
+}
+
+/* Per-tensor variants of the activation quantisation, readings R14 and R15,
+ * on the LN output of every token (LN as in oracle_ln_absmax_quant):
+ *   mode 0 (Eq.(5), per tensor):  gamma = max_{m,k} |LN_mk|
+ *          q_mk = clamp(rne(LN_mk * Q_b / gamma), -127, 127)
+ *   mode 1 (Eq.(6)):              eta = min_{m,k} LN_mk,  gamma = max_{m,k} (LN_mk - eta)
+ *          q_mk = clamp(rne((LN_mk - eta) * Q_b / gamma), 0, 127)
+ * gamma_out[m] = gamma for every token (the forward's rescale reads it per
+ * token); eta_out (may be NULL) receives eta (0 in mode 0); pre (may be
+ * NULL) the unrounded values. */
+void oracle_ln_quant_tensor(const uint16_t* x, int64_t M, int64_t K, double eps, int mode,
+                            int8_t* xq, double* gamma_out, double* eta_out, double* pre)
+{
+    const double Qb = 128.0;
+    if (eta_out) *eta_out = 0.0;
+    if (M <= 0 || K <= 0) return;
+    double* ln = (double*)malloc((size_t)(M * K) * sizeof(double));
+    if (!ln) return;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * K;
+        double sum = 0.0;
+        for (int64_t k = 0; k < K; ++k) sum += bf16_value(row[k]);
+        double mu = sum / (double)K;
+        double sq = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double d = bf16_value(row[k]) - mu;
+            sq += d * d;
+        }
+        double root = sqrt(sq / (double)K + eps);
+        for (int64_t k = 0; k < K; ++k) ln[m * K + k] = (bf16_value(row[k]) - mu) / root;
+    }
+    double eta = 0.0, gamma = 0.0;
+    if (mode == 1) {
+        eta = INFINITY;
+        for (int64_t i = 0; i < M * K; ++i)
+            if (ln[i] < eta) eta = ln[i];
+        for (int64_t i = 0; i < M * K; ++i)
+            if (ln[i] - eta > gamma) gamma = ln[i] - eta;
+    } else {
+        for (int64_t i = 0; i < M * K; ++i)
+            if (fabs(ln[i]) > gamma) gamma = fabs(ln[i]);
+    }
+    for (int64_t i = 0; i < M * K; ++i) {
+        double v = 0.0, r = 0.0;
+        if (gamma != 0.0) {
+            v = (mode == 1 ? ln[i] - eta : ln[i]) * Qb / gamma;
+            r = nearbyint(v);
+        }
+        if (r > 127.0) r = 127.0;
+        if (r < (mode == 1 ? 0.0 : -127.0)) r = (mode == 1 ? 0.0 : -127.0);
+        xq[i] = (int8_t)r;
+        if (pre) pre[i] = v;
+    }
+    for (int64_t m = 0; m < M; ++m) gamma_out[m] = gamma;
+    if (eta_out) *eta_out = eta;
+    free(ln);
 }
 
 /* integer core of [BitNet] Eq.(7): acc_mj = sum_k s_jk * q_mk  (int64) */

@@ -398,6 +398,59 @@ def pin_ternary_eps_moves_the_threshold(o):
     assert p0[0, 4] == 0 and p1[0, 4] == 0
 
 
+# ---- per-tensor Eq.(5) and the non-negative Eq.(6) quantisers ---------------
+
+def pin_quant_tensor_example_d(o):
+    ex = _load("quant_tensor_example_d.json")
+    x = np.stack([_bf16_bits_of([_frac(v) for v in row]) for row in ex["x"]])
+    for mode, key in ((0, "per_tensor"), (1, "nonneg")):
+        want = ex[key]
+        xq, gamma, eta, pre = o.ln_quant_tensor(x, mode, eps=ex["ln_eps"], want_pre=True)
+        assert xq.tolist() == want["xq"], (key, xq)
+        g = float(want["gamma"])
+        assert np.all(np.abs(gamma - g) <= 4e-16 * g), (key, gamma)
+        if mode == 1:
+            assert abs(eta - float(want["eta"])) <= 4e-16 * abs(float(want["eta"])), eta
+        for got_row, want_row in zip(pre, want["pre"]):
+            for got, w in zip(got_row, want_row):
+                assert abs(got - float(w)) <= 1e-12 * 128, (key, pre)
+
+
+def pin_quant_tensor_one_token_is_per_token(o):
+    # Eq.(5) over a one-token matrix is the per-token quantiser (a separate function)
+    rng = np.random.default_rng(21)
+    x = _to_bf16_bits((rng.standard_normal((1, 700)) * 3).astype(np.float32))
+    xq_t, g_t, _ = o.ln_quant_tensor(x, 0)
+    xq_p, g_p = o.ln_absmax_quant(x)
+    assert np.array_equal(xq_t, xq_p) and np.array_equal(g_t, g_p)
+
+
+def pin_quant_tensor_widest_token_keeps_its_codes(o):
+    # the token with the largest max|LN| sets the tensor's gamma, so its codes
+    # equal its per-token codes; every other token's |codes| can only shrink
+    rng = np.random.default_rng(22)
+    x = _to_bf16_bits((rng.standard_normal((6, 384)) * np.arange(1, 7)[:, None]).astype(np.float32))
+    x[2, 5] = _to_bf16_bits(np.array([400.0], np.float32))[0]  # an outlier: token 2 is the widest
+    xq_t, g_t, _ = o.ln_quant_tensor(x, 0)
+    xq_p, g_p = o.ln_absmax_quant(x)
+    w = int(np.argmax(g_p))
+    assert w == 2 and np.all(g_t == g_p[w])
+    assert np.array_equal(xq_t[w], xq_p[w])
+    assert np.all(np.abs(xq_t.astype(int)) <= np.abs(xq_p.astype(int)))
+
+
+def pin_quant_nonneg_range(o):
+    # Eq.(6): codes in [0, 127]; the tensor's smallest LN value maps to 0 and the
+    # largest to 127 (128 clamped); gamma = max LN - min LN
+    rng = np.random.default_rng(23)
+    x = _to_bf16_bits(rng.standard_normal((5, 256)).astype(np.float32))
+    xq, gamma, eta, pre = o.ln_quant_tensor(x, 1, want_pre=True)
+    assert xq.min() == 0 and xq.max() == 127
+    i_min, i_max = np.unravel_index(np.argmin(pre), pre.shape), np.unravel_index(np.argmax(pre), pre.shape)
+    assert xq[i_min] == 0 and xq[i_max] == 127 and pre[i_min] == 0.0 and pre[i_max] == 128.0
+    assert eta < 0 < gamma[0] and np.all(gamma == gamma[0])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]
 
 

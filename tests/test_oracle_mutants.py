@@ -51,6 +51,15 @@ MUTANTS = [
     ("w1a1_and_not_xnor", "s += (int64_t)packed_sign(a, K, m, k) * (int64_t)packed_sign(b, K, j, k);",
      "s += (packed_sign(a, K, m, k) == 1 && packed_sign(b, K, j, k) == 1) ? 1 : -1;"),
     ("bf16_decode_wrong_half", "uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+    # per-tensor Eq.(5) and non-negative Eq.(6) quantisers
+    ("tensor_gamma_per_token", "            if (fabs(ln[i]) > gamma) gamma = fabs(ln[i]);",
+     "            if (fabs(ln[i]) > gamma && i < K) gamma = fabs(ln[i]);"),
+    ("nonneg_no_eta_shift", "v = (mode == 1 ? ln[i] - eta : ln[i]) * Qb / gamma;", "v = ln[i] * Qb / gamma;"),
+    ("nonneg_gamma_absmax", "            if (ln[i] - eta > gamma) gamma = ln[i] - eta;",
+     "            if (fabs(ln[i]) > gamma) gamma = fabs(ln[i]);"),
+    # (a symmetric lower clamp is not observable in mode 1: LN - eta >= 0)
+    ("nonneg_eta_first_token", "            if (ln[i] < eta) eta = ln[i];",
+     "            if (ln[i] < eta && i < K) eta = ln[i];"),
     # b1.58 ternary weights
     ("ternary_round_half_away", "double r = nearbyint((double)W[j * K + k] / (gamma + eps));",
      "double r = round((double)W[j * K + k] / (gamma + eps));"),
