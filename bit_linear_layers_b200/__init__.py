@@ -42,6 +42,11 @@ BL_OP_W1A16 = 2
 BL_OP_W1A8 = 3
 BL_OP_PACK_TERNARY = 4
 BL_OP_W158A8 = 5
+BL_OP_W1A8_EX = 6
+
+BL_W1A8_TERNARY = 1
+BL_W1A8_PER_TENSOR = 2
+BL_W1A8_NONNEG = 4
 
 # every symbol include/bitlinear.h declares, with its ctypes signature
 _i64 = ctypes.c_int64
@@ -60,6 +65,7 @@ SIGNATURES = {
     "bl_device_error": ([_p, _int, ctypes.POINTER(_int)], _int),
     "bitlinear_w1a8_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
     "bin_xnor_gemm": ([_p, _p, _p, _i64, _i64, _i64, _p], _int),
+    "bitlinear_w1a8_ex": ([_p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_uint, _p, _sz, _p, _p, _p, _p], _int),
     "bitlinear_w158a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w158a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
 }
@@ -249,6 +255,32 @@ def bitlinear_w158a8_debug(x, packed, beta, *, xq_in=None, gamma_in=None, ws=Non
         _stream(dev))
     _check("bitlinear_w158a8_debug", rc)
     return y, xq, gamma, acc
+
+
+def bitlinear_w1a8_ex(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, flags: int, *, ws=None,
+                      debug: bool = False):
+    """bitlinear_w1a8 with the page's other activation quantisers
+    (BL_W1A8_PER_TENSOR: Eq.(5) over the matrix; BL_W1A8_NONNEG: Eq.(6)) and/or
+    ternary weights (BL_W1A8_TERNARY). Returns y, or (y, xq, gamma, acc) with
+    debug=True."""
+    M, K = x.shape
+    N = packed.shape[0]
+    dev = x.device
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    extra = [None, None, None]
+    if debug:
+        extra = [torch.empty((M, K), dtype=torch.int8, device=dev), torch.empty(M, dtype=torch.float64, device=dev),
+                 torch.empty((M, N), dtype=torch.int32, device=dev)]
+    op = BL_OP_W1A8_EX if flags & (BL_W1A8_PER_TENSOR | BL_W1A8_NONNEG) else BL_OP_W1A8
+    ws, _ = _workspace(op, M, N, K, dev, ws)
+    rc = lib.bitlinear_w1a8_ex(
+        _dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
+        _dev_ptr(beta, torch.float32, "beta"), _dev_ptr(y, torch.float32, "y"), M, N, K, int(flags),
+        _dev_ptr(ws, torch.uint8, "ws"), ws.numel() if ws is not None else 0,
+        _dev_ptr(extra[0], torch.int8, "xq"), _dev_ptr(extra[1], torch.float64, "gamma"),
+        _dev_ptr(extra[2], torch.int32, "acc"), _stream(dev))
+    _check("bitlinear_w1a8_ex", rc)
+    return (y, *extra) if debug else y
 
 
 def bitlinear_w1a8_noalloc(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, *, out=None):

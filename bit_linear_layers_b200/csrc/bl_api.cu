@@ -284,10 +284,14 @@ int launch_ts(const void* act, const uint32_t* packed, int64_t M, int64_t N, int
 }
 
 // ---- W1A8 shared body -----------------------------------------------------------
-// `ternary`: packed holds b1.58 weights (two planes, K/16 words per row)
+// `ternary`: packed holds b1.58 weights (two planes, K/16 words per row).
+// `quant`: 0 per-token gamma; BL_W1A8_PER_TENSOR: Eq.(5) over the matrix;
+// BL_W1A8_NONNEG: Eq.(6) (per tensor). The per-tensor forms need the larger
+// workspace of BL_OP_W1A8_EX.
 int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
               int64_t N, int64_t K, void* ws, size_t ws_bytes, int8_t* xq_out, double* gamma_out,
-              int32_t* acc_out, const int8_t* xq_in, const double* gamma_in, bool ternary, void* stream) {
+              int32_t* acc_out, const int8_t* xq_in, const double* gamma_in, bool ternary, void* stream,
+              unsigned quant = 0u) {
   int rc = check_shape(M, N, K);
   if (rc != BL_OK) return rc;
   if (M == 0) return BL_OK;
@@ -296,7 +300,8 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
     if (!gamma_in || !aligned16(xq_in)) return BL_ERR_INVALID_ARG;
   } else {
     if (!x || !aligned16(x)) return BL_ERR_INVALID_ARG;
-    if (!ws || !aligned16(ws) || ws_bytes < bl_workspace_bytes(BL_OP_W1A8, M, N, K))
+    if (!ws || !aligned16(ws) ||
+        ws_bytes < bl_workspace_bytes(quant ? BL_OP_W1A8_EX : BL_OP_W1A8, M, N, K))
       return BL_ERR_INVALID_ARG;
   }
   rc = device_setup(nullptr);
@@ -308,8 +313,22 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
   if (!xq_in) {
     int8_t* xq_ws = static_cast<int8_t*>(ws);
     double* g_ws = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(size_t(M * K)));
-    ln_quant_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
-    if ((rc = launch_status()) != BL_OK) return rc;
+    if (!quant) {
+      ln_quant_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
+      if ((rc = launch_status()) != BL_OK) return rc;
+    } else {
+      const bool nonneg = (quant & BL_W1A8_NONNEG) != 0;
+      auto* stats = reinterpret_cast<LnTokenStats*>(reinterpret_cast<uint8_t*>(g_ws) +
+                                                    align256(size_t(M) * sizeof(double)));
+      auto* scalars = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(stats) +
+                                                align256(size_t(M) * sizeof(LnTokenStats)));
+      ln_stats_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, stats);
+      if ((rc = launch_status()) != BL_OK) return rc;
+      ln_tensor_scalars_kernel<<<1, kLnThreads, 0, s>>>(stats, M, nonneg, g_ws, scalars);
+      if ((rc = launch_status()) != BL_OK) return rc;
+      ln_quant_tensor_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, nonneg, stats, scalars, xq_ws);
+      if ((rc = launch_status()) != BL_OK) return rc;
+    }
     codes = xq_ws;
     gam = g_ws;
   }
@@ -375,6 +394,9 @@ size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case BL_OP_PACK_TERNARY: return align256(size_t(N) * 2 * sizeof(double)) + 256;
     case BL_OP_W1A8:
     case BL_OP_W158A8: return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double));
+    case BL_OP_W1A8_EX:
+      return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double)) +
+             align256(size_t(M) * sizeof(LnTokenStats)) + 256;
     default: return 0;
   }
 }
@@ -471,6 +493,15 @@ int bitlinear_w158a8(const uint16_t* x, const uint32_t* packed, const float* bet
                      int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream) {
   return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, nullptr, nullptr, nullptr, nullptr,
                    nullptr, true, stream);
+}
+
+int bitlinear_w1a8_ex(const uint16_t* x, const uint32_t* packed, const float* beta, float* y, int64_t M,
+                      int64_t N, int64_t K, unsigned flags, void* ws, size_t ws_bytes, int8_t* xq_out,
+                      double* gamma_out, int32_t* acc_out, void* stream) {
+  if (flags & ~(BL_W1A8_TERNARY | BL_W1A8_PER_TENSOR | BL_W1A8_NONNEG)) return BL_ERR_INVALID_ARG;
+  const unsigned quant = flags & (BL_W1A8_PER_TENSOR | BL_W1A8_NONNEG);
+  return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, xq_out, gamma_out, acc_out, nullptr, nullptr,
+                   (flags & BL_W1A8_TERNARY) != 0, stream, quant);
 }
 
 int bitlinear_w158a8_debug(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,

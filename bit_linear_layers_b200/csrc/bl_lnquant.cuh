@@ -170,4 +170,141 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
   }
 }
 
+// ---------------------------------------------------------------------------
+// Per-tensor variants ("BitNet b1.58" page, section 1): Eq.(5) with gamma
+// over the whole LN output of the matrix, and Eq.(6), which shifts by the
+// matrix's smallest LN value eta and scales the range max(LN - eta) onto
+// [0, Q_b] (codes 0..127). Three kernels: per-token statistics, one CTA that
+// folds them into gamma (and eta), then per-token quantisation. Codes are
+// evaluated in fp64 in the order of the formula: ln = (x - mu) / root,
+// v = (ln [- eta]) * 128 / gamma, rounded half to even and clamped.
+struct LnTokenStats {
+  double mu, root, ln_min, ln_max;  // ln_min / ln_max: the token's extreme LN values
+};
+
+__global__ void __launch_bounds__(kLnThreads) ln_stats_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                              int64_t K, LnTokenStats* __restrict__ stats) {
+  __shared__ double sh[kLnWarps];
+  __shared__ float shm[2][kLnWarps];
+  const int64_t m = blockIdx.x;
+  if (m >= M) return;  // uniform per CTA
+  const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
+  const int64_t nvec = K / 8;
+  double s0 = 0.0, s1 = 0.0;
+  float xmax = -INFINITY, xmin = INFINITY;
+  for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
+    const uint4 v = row[i];
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      s0 += bf16_to_double(h[j] & 0xFFFFu);
+      s1 += bf16_to_double(h[j] >> 16);
+      const float a = bf16_lo(h[j]), b = bf16_hi(h[j]);
+      xmax = fmaxf(xmax, fmaxf(a, b));
+      xmin = fminf(xmin, fminf(a, b));
+    }
+  }
+  xmax = warp_max(xmax);
+  xmin = -warp_max(-xmin);
+  if ((threadIdx.x & 31) == 0) {
+    shm[0][threadIdx.x >> 5] = xmax;
+    shm[1][threadIdx.x >> 5] = xmin;
+  }
+  const double mu = ln_block_sum(s0 + s1, sh) / static_cast<double>(K);
+  xmax = shm[0][0];
+  xmin = shm[1][0];
+#pragma unroll
+  for (int w = 1; w < kLnWarps; ++w) {
+    xmax = fmaxf(xmax, shm[0][w]);
+    xmin = fminf(xmin, shm[1][w]);
+  }
+  double q0 = 0.0, q1 = 0.0;
+  for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
+    const uint4 v = row[i];
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const double d0 = bf16_to_double(h[j] & 0xFFFFu) - mu;
+      const double d1 = bf16_to_double(h[j] >> 16) - mu;
+      q0 = fma(d0, d0, q0);
+      q1 = fma(d1, d1, q1);
+    }
+  }
+  const double sq = ln_block_sum(q0 + q1, sh);
+  if (threadIdx.x == 0) {
+    const double root = sqrt(sq / static_cast<double>(K) + kLnEps);
+    // (x - mu) / root is monotonic in x: the token's extremes come from x_min and x_max
+    stats[m] = LnTokenStats{mu, root, (static_cast<double>(xmin) - mu) / root,
+                            (static_cast<double>(xmax) - mu) / root};
+  }
+}
+
+// One CTA: gamma (and eta) over all tokens; gamma_out[m] = gamma for every m,
+// scalars[0] = gamma, scalars[1] = eta (0 for Eq.(5)).
+__global__ void __launch_bounds__(kLnThreads) ln_tensor_scalars_kernel(const LnTokenStats* __restrict__ stats,
+                                                                       int64_t M, bool nonneg,
+                                                                       double* __restrict__ gamma_out,
+                                                                       double* __restrict__ scalars) {
+  __shared__ double sh_a[kLnWarps], sh_b[kLnWarps];
+  double amax = 0.0, lmin = INFINITY, lmax = -INFINITY;
+  for (int64_t m = threadIdx.x; m < M; m += kLnThreads) {
+    const LnTokenStats t = stats[m];
+    amax = fmax(amax, fmax(fabs(t.ln_min), fabs(t.ln_max)));
+    lmin = fmin(lmin, t.ln_min);
+    lmax = fmax(lmax, t.ln_max);
+  }
+  amax = warp_max(amax);
+  lmax = warp_max(lmax);
+  lmin = -warp_max(-lmin);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sh_a[w] = nonneg ? lmax : amax;
+    sh_b[w] = lmin;
+  }
+  __syncthreads();
+  double g = sh_a[0], e = sh_b[0];
+  for (int i = 1; i < kLnWarps; ++i) {
+    g = fmax(g, sh_a[i]);
+    e = fmin(e, sh_b[i]);
+  }
+  // Eq.(6): gamma = max (LN - eta) = max LN - eta (the rounded difference is monotonic)
+  const double eta = nonneg ? e : 0.0;
+  const double gamma = nonneg ? g - eta : g;
+  for (int64_t m = threadIdx.x; m < M; m += kLnThreads) gamma_out[m] = gamma;
+  if (threadIdx.x == 0) {
+    scalars[0] = gamma;
+    scalars[1] = eta;
+  }
+}
+
+__global__ void __launch_bounds__(kLnThreads) ln_quant_tensor_kernel(const uint16_t* __restrict__ x, int64_t M,
+                                                                     int64_t K, bool nonneg,
+                                                                     const LnTokenStats* __restrict__ stats,
+                                                                     const double* __restrict__ scalars,
+                                                                     int8_t* __restrict__ xq) {
+  const int64_t m = blockIdx.x;
+  if (m >= M) return;
+  const LnTokenStats t = stats[m];
+  const double gamma = scalars[0], eta = scalars[1];
+  const double lo = nonneg ? 0.0 : -127.0;
+  const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
+  uint2* out = reinterpret_cast<uint2*>(xq + m * K);
+  for (int64_t i = threadIdx.x; i < K / 8; i += kLnThreads) {
+    const uint4 v = row[i];
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+    uint32_t codes[2] = {0u, 0u};
+    if (gamma != 0.0) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t b16 = (h[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+        const double ln = (bf16_to_double(b16) - t.mu) / t.root;
+        const double val = (nonneg ? ln - eta : ln) * 128.0 / gamma;
+        const int q = static_cast<int>(fmin(fmax(rint(val), lo), 127.0));
+        codes[j >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (j & 3));
+      }
+    }
+    out[i] = make_uint2(codes[0], codes[1]);
+  }
+}
+
 }  // namespace bl

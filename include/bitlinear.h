@@ -66,6 +66,7 @@ extern "C" {
 #define BL_OP_W1A8 3
 #define BL_OP_PACK_TERNARY 4
 #define BL_OP_W158A8 5
+#define BL_OP_W1A8_EX 6 /* bitlinear_w1a8_ex with a per-tensor quantiser */
 
 /* Library ABI version (this header: 1). */
 int bl_abi_version(void);
@@ -183,6 +184,32 @@ int bitlinear_w158a8_debug(const uint16_t* x, const uint32_t* packed, const floa
                            int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes,
                            int8_t* xq_out, double* gamma_out, int32_t* acc_out,
                            const int8_t* xq_in, const double* gamma_in, void* stream);
+
+/*
+ * bitlinear_w1a8_ex -- bitlinear_w1a8 / bitlinear_w158a8 with the other
+ * activation quantisers of the "BitNet b1.58" page, section 1:
+ *   BL_W1A8_PER_TENSOR  Eq.(5) as printed, gamma = ||LN(x)||_inf over the
+ *                       whole M x K matrix (shared by every token); codes
+ *                       clamp(rne(LN * 128 / gamma), -127, 127).
+ *   BL_W1A8_NONNEG      Eq.(6), for activations before a nonlinearity:
+ *                       eta = smallest LN value of the matrix, gamma =
+ *                       max(LN - eta), codes clamp(rne((LN - eta) * 128 /
+ *                       gamma), 0, 127); the output is Eq.(7) as printed,
+ *                       y = acc * beta * gamma / 128 (no eta term appears on
+ *                       the page). Implies per tensor.
+ *   BL_W1A8_TERNARY     packed holds b1.58 ternary weights (BL_PACK_TERNARY).
+ * With neither quantiser flag this is bitlinear_w1a8 (or w158a8). Codes are
+ * decided in fp64 in the order of the formula. ws: bl_workspace_bytes(
+ * BL_OP_W1A8_EX, M, N, K) bytes for the per-tensor forms (else BL_OP_W1A8).
+ * xq_out [M x K], gamma_out [M] (the shared gamma, repeated) and acc_out
+ * [M x N] may be NULL.
+ */
+#define BL_W1A8_TERNARY 1u
+#define BL_W1A8_PER_TENSOR 2u
+#define BL_W1A8_NONNEG 4u
+int bitlinear_w1a8_ex(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
+                      int64_t M, int64_t N, int64_t K, unsigned flags, void* ws, size_t ws_bytes,
+                      int8_t* xq_out, double* gamma_out, int32_t* acc_out, void* stream);
 
 /*
  * bin_xnor_gemm -- W1A1: products of two +-1 matrices ("BitNet-Transformers"

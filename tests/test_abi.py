@@ -49,6 +49,8 @@ def test_workspace_sizes():
     ws = bl.workspace_bytes(bl.BL_OP_W1A8, 512, 5632, 2048)
     assert ws >= 512 * 2048 + 512 * 8 and ws % 256 == 0
     assert bl.workspace_bytes(bl.BL_OP_W1A8, -1, 1, 128) == 0
+    ex = bl.workspace_bytes(bl.BL_OP_W1A8_EX, 512, 5632, 2048)
+    assert ex >= ws + 512 * 32 + 16 and ex % 256 == 0
 
 
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case below fails validation
@@ -74,6 +76,12 @@ def test_null_and_misaligned_pointers_rejected():
     assert bl.lib.bitlinear_w1a8(FAKE, FAKE, None, FAKE, 1, 128, 128, FAKE, 1 << 20, None) == -1
     # workspace too small
     assert bl.lib.bitlinear_w1a8(FAKE, FAKE, FAKE, FAKE, 4, 128, 128, FAKE, 16, None) == -1
+    # unknown quantiser flag; a per-tensor quantiser given the per-token workspace
+    assert bl.lib.bitlinear_w1a8_ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 128, 8, FAKE, 1 << 20,
+                                    None, None, None, None) == -1
+    small = bl.workspace_bytes(bl.BL_OP_W1A8, 4, 128, 128)
+    assert bl.lib.bitlinear_w1a8_ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 128, bl.BL_W1A8_NONNEG, FAKE, small,
+                                    None, None, None, None) == -1
     assert bl.lib.bin_pack(FAKE, 128, 128, 7, FAKE, FAKE, FAKE, None, 0, None) == -1
     assert bl.lib.bin_pack(FAKE, 128, 128, bl.BL_PACK_BITNET, FAKE, FAKE, FAKE, None, 0, None) == -1
     assert bl.lib.bin_pack(FAKE, 128, 96, bl.BL_PACK_FBI, FAKE, FAKE, None, None, 0, None) == -2
