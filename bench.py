@@ -384,7 +384,7 @@ class W1A8(Workload):
                 p, _, b = bl.bin_pack(W, bl.BL_PACK_BITNET)
                 del W
                 x = synthetic.laplace_channel_activations(M, K, seed=seed, device=dev)
-                ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W1A8, M, N, K), dtype=torch.uint8, device=dev)
+                ws = torch.empty(bl.workspace_bytes(self.ws_op(bl), M, N, K), dtype=torch.uint8, device=dev)
                 y = torch.empty((M, N), dtype=torch.float32, device=dev)
                 layers.append((x, p, b, ws, y))
             self.copies.append(layers)
@@ -393,14 +393,20 @@ class W1A8(Workload):
         self.h2d = sum(M * K * 2 for M, K, N in self.SHAPES)
         self.d2h = sum(M * N * 4 for M, K, N in self.SHAPES)
 
+    def ws_op(self, bl):
+        return bl.BL_OP_W1A8
+
+    def call(self, x, p, b, ws, y):
+        self.bl.bitlinear_w1a8(x, p, b, out=y, ws=ws)
+
     def step(self, i):
         for x, p, b, ws, y in self.copies[i % self.rotate]:
-            self.bl.bitlinear_w1a8(x, p, b, out=y, ws=ws)
+            self.call(x, p, b, ws, y)
 
     def e2e_step(self, i):
         for (x, p, b, ws, y), xh, yh in zip(self.copies[i % self.rotate], self.xh, self.yh):
             x.copy_(xh, non_blocking=True)
-            self.bl.bitlinear_w1a8(x, p, b, out=y, ws=ws)
+            self.call(x, p, b, ws, y)
             yh.copy_(y, non_blocking=True)
 
     # oracle: token 0 through output columns [0, 1024) of both projections
@@ -463,15 +469,8 @@ class W158A8(W1A8):
         self.h2d = sum(M * K * 2 for M, K, N in self.SHAPES)
         self.d2h = sum(M * N * 4 for M, K, N in self.SHAPES)
 
-    def step(self, i):
-        for x, p, b, ws, y in self.copies[i % self.rotate]:
-            self.bl.bitlinear_w158a8(x, p, b, out=y, ws=ws)
-
-    def e2e_step(self, i):
-        for (x, p, b, ws, y), xh, yh in zip(self.copies[i % self.rotate], self.xh, self.yh):
-            x.copy_(xh, non_blocking=True)
-            self.bl.bitlinear_w158a8(x, p, b, out=y, ws=ws)
-            yh.copy_(y, non_blocking=True)
+    def call(self, x, p, b, ws, y):
+        self.bl.bitlinear_w158a8(x, p, b, out=y, ws=ws)
 
     def oracle_setup(self):
         import oracle as oracle_pkg
@@ -491,6 +490,56 @@ class W158A8(W1A8):
     def oracle_call(self):
         for x, p, gamma_w, K in self.olayers:
             self.o.w158a8(x, p, gamma_w, K)
+
+
+class W1A8Tensor(W1A8):
+    """The W1A8 workload with the per-tensor absmax quantiser (Eq.(5) of the
+    "BitNet b1.58" page with gamma over the whole LN output matrix): token
+    statistics, one gamma, then quantisation, before the same int8 GEMM. The
+    non-negative Eq.(6) form runs the same kernels with one flag."""
+    name = "w1a8_tensor"
+    metric = "BitLinear W1A8 TOP/s, per-tensor activation gamma (1.3B shapes, 512 tokens)"
+    kernel = ("ln_stats_kernel + ln_tensor_scalars_kernel + ln_quant_tensor_kernel + gemm_ts_kernel<1,*> "
+              "(one call; time includes LN + quantisation)")
+    traffic_file = None
+    launches_per_step = 8
+
+    def __init__(self):
+        super().__init__()
+        self.config = dict(self.config)
+        self.config["workload"] = ("BitNet BitLinear W1A8, 512 tokens, 1.3B shapes 2048->5632 then 5632->2048, "
+                                   "per-tensor activation gamma")
+
+    def ws_op(self, bl):
+        return bl.BL_OP_W1A8_EX
+
+    def call(self, x, p, b, ws, y):
+        self.bl.bitlinear_w1a8_ex(x, p, b, self.bl.BL_W1A8_PER_TENSOR, out=y, ws=ws)
+
+    def oracle_setup(self):
+        import oracle as oracle_pkg
+        from bit_linear_layers_b200 import synthetic
+        self.o = oracle_pkg.get()
+        self.olayers, ops = [], 0.0
+        for s, (M, K, N) in enumerate(self.SHAPES):
+            W = synthetic.weights(N, K, seed=4 + 10 * s, mean=0.001).numpy()
+            p, _, beta = self.o.pack_bitnet(W)
+            x = synthetic.bf16_bits(synthetic.laplace_channel_activations(M, K, seed=4 + 10 * s))
+            self.olayers.append((x, p, beta, K))
+            ops += 2.0 * K * self.ORACLE_COLS
+        self.oracle_sample = ("LN + per-tensor quantisation of all 512 tokens (gamma needs them all), then token 0 "
+                              "through output columns 0..1023 of both projections per call (single-threaded C "
+                              "oracle, fp64/int64)")
+        return ops
+
+    def oracle_call(self):
+        import numpy as np
+        js = np.arange(self.ORACLE_COLS)
+        ms = np.zeros_like(js)
+        for x, p, beta, K in self.olayers:
+            xq, gamma, _ = self.o.ln_quant_tensor(x, 0)
+            acc = self.o.w1a8_acc_at(xq, p, K, ms, js)
+            self.o.w1a8_rescale(acc.reshape(1, -1), gamma[:1], beta)
 
 
 class W1A1(Workload):
@@ -575,7 +624,7 @@ class W1A1(Workload):
             self.o.w1a1(a, b, K)
 
 
-WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8, W158A8, W1A1)}
+WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8, W158A8, W1A8Tensor, W1A1)}
 
 
 # ----------------------------------------------------------------------------- ours

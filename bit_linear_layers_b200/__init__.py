@@ -257,8 +257,8 @@ def bitlinear_w158a8_debug(x, packed, beta, *, xq_in=None, gamma_in=None, ws=Non
     return y, xq, gamma, acc
 
 
-def bitlinear_w1a8_ex(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, flags: int, *, ws=None,
-                      debug: bool = False):
+def bitlinear_w1a8_ex(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, flags: int, *, out=None,
+                      ws=None, debug: bool = False):
     """bitlinear_w1a8 with the page's other activation quantisers
     (BL_W1A8_PER_TENSOR: Eq.(5) over the matrix; BL_W1A8_NONNEG: Eq.(6)) and/or
     ternary weights (BL_W1A8_TERNARY). Returns y, or (y, xq, gamma, acc) with
@@ -266,7 +266,7 @@ def bitlinear_w1a8_ex(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor,
     M, K = x.shape
     N = packed.shape[0]
     dev = x.device
-    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=dev)
     extra = [None, None, None]
     if debug:
         extra = [torch.empty((M, K), dtype=torch.int8, device=dev), torch.empty(M, dtype=torch.float64, device=dev),

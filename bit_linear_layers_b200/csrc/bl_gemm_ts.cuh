@@ -67,7 +67,6 @@ struct TsCfg {
   static constexpr int ATOM_BYTES = T * 128;
   static constexpr int X_UNIT_BYTES = ATOMS * ATOM_BYTES;
   static constexpr int BITS_BYTES = ROWS * 16 * PLANES;         // one 128-k sign stage
-  static constexpr int SB = 4;                                  // sign stages in shared memory
   static constexpr int OUT_ELEM = KIND == 0 ? 2 : 4;            // y element bytes
   // the output tile is staged in shared memory and written by bulk tensor
   // stores: the whole tile at once when it fits in 64 KB, else one 128-row
@@ -79,6 +78,12 @@ struct TsCfg {
   static constexpr int IN_STRIDE = T + 4;
   // staged output [T][STAGE_COLS], or the split-K inbox [S][ROWS/S][IN_STRIDE] of 4-byte partials
   static constexpr int OUT_BYTES = SPLIT ? ROWS * IN_STRIDE * 4 : (STAGE_OUT ? STAGE_COLS * T * OUT_ELEM : 0);
+  // sign stages in shared memory. A row tile's signs come from HBM on first
+  // touch, and the stages in flight must cover that latency: int8 problems
+  // (one unit is only 4-8 MMAs) take 16 stages unless that would leave fewer
+  // than four activation units; the bf16 configurations keep 4.
+  static constexpr int SX_IF_DEEP = (220 * 1024 - OUT_BYTES - 16 * BITS_BYTES) / X_UNIT_BYTES;
+  static constexpr int SB = (KIND != 0 && SX_IF_DEEP >= 4) ? 16 : 4;
   static constexpr int SX_FIT = (220 * 1024 - OUT_BYTES - SB * BITS_BYTES) / X_UNIT_BYTES;
   static constexpr int SX = SX_FIT > 8 ? 8 : SX_FIT;           // activation units in flight
   static constexpr int X_RING = SX * X_UNIT_BYTES;
@@ -232,6 +237,23 @@ __device__ __forceinline__ void expand16_ternary(uint32_t plus, uint32_t minus, 
   }
 }
 
+// Shared-memory accesses by address. The epilogue's loads and stores take no
+// "memory" clobber: as volatile asm they stay ordered with the barrier waits
+// and fences (also volatile asm) around them, and may overlap the plain
+// global stores in between.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t* v) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "r"(addr));
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v));
+}
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v));
+}
 __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, const uint32_t* v, uint32_t remote_bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
                    remote_addr),
@@ -492,7 +514,9 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
         row_alpha[rr] = j < N ? alpha[j] : 0.f;
       }
     }
-    if (threadIdx.x == 128) mbar_arrive_expect_tx(smem_u32(&inbox_bar), ROWS * T * 4);
+    // partials of the rows this CTA owns go to its own inbox with plain shared
+    // stores; only the other S - 1 CTAs' partials are counted on the barrier
+    if (threadIdx.x == 128) mbar_arrive_expect_tx(smem_u32(&inbox_bar), (S - 1) * rows_per * T * 4);
     asm volatile("barrier.cluster.wait;" ::: "memory");  // every inbox barrier is initialised
     // warp-uniform outcome: the TMEM loads below are warp-collective
     const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&d_full), 0, kWhereGemmEpilogue));
@@ -503,7 +527,8 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
       const uint32_t owner = static_cast<uint32_t>(jl / rows_per);
       const uint32_t slot0 =
           smem_u32(inbox + (static_cast<int>(rank) * rows_per + jl % rows_per) * IN_STRIDE * 4);
-      const uint32_t rslot = ts_map_rank(slot0, owner);
+      const bool local = owner == rank;
+      const uint32_t rslot = local ? slot0 : ts_map_rank(slot0, owner);
       const uint32_t rbar = ts_map_rank(smem_u32(&inbox_bar), owner);
 #pragma unroll 1
       for (int cc = 0; cc < T / 32; ++cc) {
@@ -511,25 +536,33 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
         __syncwarp();
         tmem_ld_32x32b_x32(tmem + blk * T + cc * 32 + (static_cast<uint32_t>(q * 32) << 16), r);
         tmem_wait_ld();
+        if (local) {
 #pragma unroll
-        for (int v = 0; v < 8; ++v) st_async_v4(rslot + (cc * 32 + v * 4) * 4, r + v * 4, rbar);
+          for (int v = 0; v < 8; ++v) st_shared_v4(rslot + (cc * 32 + v * 4) * 4, r + v * 4);
+        } else {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) st_async_v4(rslot + (cc * 32 + v * 4) * 4, r + v * 4, rbar);
+        }
       }
     }
-    epilogue_bar();  // tok_scale / row_alpha are written
-    // owner: add the S partials of its rows in rank order, then scale and store;
-    // a thread takes one row and four consecutive tokens (the padded inbox rows
-    // make the 16-byte reads of a warp conflict-free; lanes = consecutive rows,
-    // so each output store of a warp is contiguous)
+    epilogue_bar();  // tok_scale / row_alpha and the local partials are written
+    // owner: add the S partials of its rows in rank order, then scale and store.
+    // A thread keeps one row (rows_per is 16, 32 or 64, so lanes are consecutive
+    // rows and each output store of a warp is contiguous) and steps over groups
+    // of four tokens; the padded inbox rows make the 16-byte reads conflict-free.
     if (mbar_wait(smem_u32(&inbox_bar), 0, kWhereGemmEpilogue)) {
-      for (int e = et; e < rows_per * (T / 4); e += 128) {
-        const int rr = e % rows_per, tq = e / rows_per;
-        const int j = w0 + static_cast<int>(rank) * rows_per + rr;
-        if (j >= N) continue;
+      const int rows_shift = __ffs(rows_per) - 1;
+      const int rr = et & (rows_per - 1);
+      const int j = w0 + static_cast<int>(rank) * rows_per + rr;
+      const float arow = (KIND == 0) ? row_alpha[rr] : 0.f;
+      const uint32_t in0 = smem_u32(inbox + rr * IN_STRIDE * 4);
+      constexpr int kQuads = T / 4;
+      for (int tq = et >> rows_shift; j < N && tq < kQuads; tq += 128 >> rows_shift) {
         uint32_t sum[4] = {0u, 0u, 0u, 0u};
         float fsum[4] = {0.f, 0.f, 0.f, 0.f};
         for (int src = 0; src < S; ++src) {
-          const uint4 v = *reinterpret_cast<const uint4*>(inbox + ((src * rows_per + rr) * IN_STRIDE + 4 * tq) * 4);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          uint32_t w[4];
+          ld_shared_v4(in0 + (src * rows_per * IN_STRIDE + 4 * tq) * 4, w);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             if (KIND == 0)
@@ -538,17 +571,37 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
               sum[i] += w[i];  // two's complement: exact int32 sum
           }
         }
+        const int m0 = t0 + 4 * tq;
+        if (KIND == 0) {
+          uint16_t* yp = reinterpret_cast<uint16_t*>(y) + static_cast<int64_t>(m0) * N + j;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tt = 4 * tq + i, m = t0 + tt;
-          if (m >= M) continue;
-          const int64_t o = static_cast<int64_t>(m) * N + j;
-          if (KIND == 0) {
-            reinterpret_cast<uint16_t*>(y)[o] = float_to_bf16_bits(fsum[i] * row_alpha[rr]);
+          for (int i = 0; i < 4; ++i, yp += N)
+            if (m0 + i < M) *yp = float_to_bf16_bits(fsum[i] * arow);
+        } else {
+          float out[4];
+          const bool fast = w1a8_fast_ok(static_cast<int32_t>(sum[0])) && w1a8_fast_ok(static_cast<int32_t>(sum[1])) &&
+                            w1a8_fast_ok(static_cast<int32_t>(sum[2])) && w1a8_fast_ok(static_cast<int32_t>(sum[3]));
+          if (fast) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) out[i] = w1a8_output_fast(static_cast<int32_t>(sum[i]), tok_scale[4 * tq + i]);
           } else {
-            const int32_t acc = static_cast<int32_t>(sum[i]);
-            reinterpret_cast<float*>(y)[o] = w1a8_output(acc, tok_scale[tt]);
-            if (acc_out) acc_out[o] = acc;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) out[i] = w1a8_output(static_cast<int32_t>(sum[i]), tok_scale[4 * tq + i]);
+          }
+          float* yp = reinterpret_cast<float*>(y) + static_cast<int64_t>(m0) * N + j;
+          if (m0 + 4 <= M) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i, yp += N) *yp = out[i];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i, yp += N)
+              if (m0 + i < M) *yp = out[i];
+          }
+          if (acc_out) {
+            int32_t* ap = acc_out + static_cast<int64_t>(m0) * N + j;
+#pragma unroll
+            for (int i = 0; i < 4; ++i, ap += N)
+              if (m0 + i < M) *ap = static_cast<int32_t>(sum[i]);
           }
         }
       }
@@ -611,15 +664,22 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
               if (lane == 0) mbar_arrive(smem_u32(&d_empty));
             }
             const int ml0 = cc * 32;
+            // rows past N and tokens past M are skipped; the tests are hoisted
+            // out of the element loops, which stay free of branches
+            const bool chunk_full = jv && t0 + ml0 + 32 <= M;
             if (KIND == 0) {
+              uint16_t v[32];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int m = t0 + ml0 + i;
-                const uint16_t v = float_to_bf16_bits(__uint_as_float(r[i]) * a);
-                if (staged)
-                  reinterpret_cast<uint16_t*>(stage_out)[(ml0 + i) * C::STAGE_COLS + js] = v;
-                else if (jv && m < M)
-                  reinterpret_cast<uint16_t*>(y)[static_cast<int64_t>(m) * N + j] = v;
+              for (int i = 0; i < 32; ++i) v[i] = float_to_bf16_bits(__uint_as_float(r[i]) * a);
+              if (staged) {
+                const uint32_t so = smem_u32(stage_out) + (ml0 * C::STAGE_COLS + js) * 2;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) st_shared_u16(so + i * C::STAGE_COLS * 2, v[i]);
+              } else if (jv) {
+                uint16_t* yp = reinterpret_cast<uint16_t*>(y) + static_cast<int64_t>(t0 + ml0) * N + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i, yp += N)
+                  if (chunk_full || t0 + ml0 + i < M) *yp = v[i];
               }
             } else {
               // the fp32 form covers the chunk unless some |acc| is very large
@@ -636,14 +696,25 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = w1a8_output(static_cast<int32_t>(r[i]), tok_scale[ml0 + i]);
               }
+              if (staged) {
+                const uint32_t so = smem_u32(stage_out) + (ml0 * C::STAGE_COLS + js) * 4;
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int m = t0 + ml0 + i;
-                if (staged)
-                  reinterpret_cast<float*>(stage_out)[(ml0 + i) * C::STAGE_COLS + js] = v[i];
-                else if (jv && m < M)
-                  reinterpret_cast<float*>(y)[static_cast<int64_t>(m) * N + j] = v[i];
-                if (acc_out && jv && m < M) acc_out[static_cast<int64_t>(m) * N + j] = static_cast<int32_t>(r[i]);
+                for (int i = 0; i < 32; ++i) st_shared_f32(so + i * C::STAGE_COLS * 4, v[i]);
+              } else if (chunk_full) {
+                float* yp = reinterpret_cast<float*>(y) + static_cast<int64_t>(t0 + ml0) * N + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i, yp += N) *yp = v[i];
+              } else if (jv) {
+                float* yp = reinterpret_cast<float*>(y) + static_cast<int64_t>(t0 + ml0) * N + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i, yp += N)
+                  if (t0 + ml0 + i < M) *yp = v[i];
+              }
+              if (acc_out && jv) {
+                int32_t* ap = acc_out + static_cast<int64_t>(t0 + ml0) * N + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i, ap += N)
+                  if (t0 + ml0 + i < M) *ap = static_cast<int32_t>(r[i]);
               }
             }
           }
