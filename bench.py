@@ -813,6 +813,33 @@ def secondary_llama7b(dev, peaks):
                                    "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                    "launches_per_step": 224}
         del gph
+        if B == 1:
+            # the same chain as one stacked launch: 128 levels (q,k,v | o | gate,up | down per layer)
+            levels = []
+            for i, mats in enumerate(layers):
+                cur = x.reshape(-1) if i == 0 else h.reshape(-1)
+                levels.append((cur, [(mats[0][0], mats[0][1], q), (mats[1][0], mats[1][1], k),
+                                     (mats[2][0], mats[2][1], v)]))
+                levels.append((v.reshape(-1), [(mats[3][0], mats[3][1], o)]))
+                levels.append((o.reshape(-1), [(mats[4][0], mats[4][1], g), (mats[5][0], mats[5][1], u)]))
+                levels.append((u.reshape(-1), [(mats[6][0], mats[6][1], h)]))
+            stack = bl.W1A16Stack(levels)
+            for _ in range(3):
+                stack.run()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                stack.run()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            res["decode_batch1_stack"] = {
+                "ms_per_token_step": ms, "tok_s": 1.0 / (ms * 1e-3),
+                "packed_GB_per_s": packed_bytes / (ms * 1e-3) / 1e9,
+                "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "launches_per_step": 1, "call": "bin_linear_w1a16_stack (one zero-fill + one persistent kernel)"}
     # prefill: 4096 tokens through every linear (not chained: fixed inputs)
     T = 4096
     x4 = synthetic.activations(T, 4096, seed=78, device=dev)

@@ -43,6 +43,7 @@ BL_OP_W1A8 = 3
 BL_OP_PACK_TERNARY = 4
 BL_OP_W158A8 = 5
 BL_OP_W1A8_EX = 6
+BL_OP_W1A16_STACK = 7
 
 BL_W1A8_TERNARY = 1
 BL_W1A8_PER_TENSOR = 2
@@ -53,6 +54,18 @@ _i64 = ctypes.c_int64
 _p = ctypes.c_void_p
 _int = ctypes.c_int
 _sz = ctypes.c_size_t
+class StackJob(ctypes.Structure):
+    """bl_stack_job: one linear of a stack level."""
+    _fields_ = [("packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("N", ctypes.c_int64)]
+
+
+class StackLevel(ctypes.Structure):
+    """bl_stack_level: one input vector and the linears that read it."""
+    _fields_ = [("x", ctypes.c_void_p), ("K", ctypes.c_int64), ("first_job", ctypes.c_int32),
+                ("num_jobs", ctypes.c_int32)]
+
+
 SIGNATURES = {
     "bl_abi_version": ([], _int),
     "bl_status_string": ([_int], ctypes.c_char_p),
@@ -65,6 +78,7 @@ SIGNATURES = {
     "bl_device_error": ([_p, _int, ctypes.POINTER(_int)], _int),
     "bitlinear_w1a8_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
     "bin_xnor_gemm": ([_p, _p, _p, _i64, _i64, _i64, _p], _int),
+    "bin_linear_w1a16_stack": ([_p, _int, _p, _int, _p, _sz, _p], _int),
     "bitlinear_w1a8_ex": ([_p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_uint, _p, _sz, _p, _p, _p, _p], _int),
     "bitlinear_w158a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w158a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
@@ -178,6 +192,46 @@ def bin_linear_w1a16(x: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor,
         rc = lib.bin_linear_w1a16(*args, _stream(x.device))
         _check("bin_linear_w1a16", rc)
     return out
+
+
+class W1A16Stack:
+    """A stack of single-token FBI-linear layers run by bin_linear_w1a16_stack.
+
+    `levels` is a list of (x, linears), x a bf16 [K] (or [1, K]) device tensor
+    and linears a list of (packed, alpha, y) with y a bf16 [N] (or [1, N])
+    tensor the call writes. A level may read any y of an earlier level. The
+    descriptor arrays are built once; run() enqueues the whole stack on the
+    current stream."""
+
+    def __init__(self, levels, *, ws=None):
+        jobs, lvls = [], []
+        self._keep = []
+        dev = None
+        for x, linears in levels:
+            K = x.shape[-1]
+            if x.numel() != K:
+                raise ValueError("stack inputs are single vectors")
+            dev = x.device
+            lvls.append(StackLevel(_dev_ptr(x, torch.bfloat16, "x"), K, len(jobs), len(linears)))
+            for packed, alpha, y in linears:
+                N = packed.shape[0]
+                if y.numel() != N or packed.shape[1] * 32 != K:
+                    raise ValueError("linear shapes do not match the level input")
+                jobs.append(StackJob(_dev_ptr(packed, torch.int32, "packed"), _dev_ptr(alpha, torch.float32, "alpha"),
+                                     _dev_ptr(y, torch.bfloat16, "y"), N))
+                self._keep += [packed, alpha, y]
+            self._keep.append(x)
+        self._levels = (StackLevel * max(len(lvls), 1))(*lvls)
+        self._jobs = (StackJob * max(len(jobs), 1))(*jobs)
+        self.num_levels, self.num_jobs = len(lvls), len(jobs)
+        self.device = dev
+        self.ws, self.ws_bytes = _workspace(BL_OP_W1A16_STACK, 0, 0, 0, dev, ws)
+
+    def run(self):
+        rc = lib.bin_linear_w1a16_stack(ctypes.byref(self._levels), self.num_levels, ctypes.byref(self._jobs),
+                                        self.num_jobs, _dev_ptr(self.ws, torch.uint8, "ws"), self.ws.numel(),
+                                        _stream(self.device))
+        _check("bin_linear_w1a16_stack", rc)
 
 
 def bitlinear_w1a8(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, *, out=None, ws=None):

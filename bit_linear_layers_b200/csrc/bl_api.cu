@@ -15,6 +15,7 @@
 #include "bl_gemm_ts.cuh"
 #include "bl_gemv.cuh"
 #include "bl_gemv_lut.cuh"
+#include "bl_gemv_stack.cuh"
 #include "bl_lnquant.cuh"
 #include "bl_pack.cuh"
 #include "bl_xnor.cuh"
@@ -39,6 +40,8 @@ struct DeviceState {
   // can be resident at once: clusters must fit inside a GPC, so this is
   // below num_sms / S (on B200: 74 / 33 / 15)
   int cluster_cap[9] = {};
+  // clusters of 8 stacked-decode CTAs that can be resident at once
+  int stack_clusters = 0;
 };
 DeviceState g_devices[kMaxDevices];
 
@@ -80,8 +83,28 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<1>, 1 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<2>, 2 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
-              set_ts_smem<0>() && set_ts_smem<1>() && set_ts_smem<2>();
+              set_ts_smem<0>() && set_ts_smem<1>() && set_ts_smem<2>() &&
+              set_smem(gemv_w1a16_stack_kernel, kStackPages * kLutPageBytes);
     if (!ok) cudaGetLastError();
+    {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kStackCluster, 1, 1);
+      cfg.blockDim = dim3(kLutThreads, 1, 1);
+      cfg.dynamicSmemBytes = kStackPages * kLutPageBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kStackCluster;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemv_w1a16_stack_kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = 0;  // the stacked decode then reports BL_ERR_CUDA
+      }
+      st.stack_clusters = n;
+    }
     for (int S : {2, 4, 8}) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(static_cast<unsigned>(S), 1, 1);
@@ -105,6 +128,15 @@ int device_setup(int* num_sms) {
   });
   if (num_sms) *num_sms = st.num_sms;
   return st.status;
+}
+
+int stack_cluster_capacity() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 0;
+  }
+  return g_devices[dev].stack_clusters;
 }
 
 // co-resident cluster capacity of the current device for clusters of S GEMM CTAs
@@ -397,6 +429,7 @@ size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case BL_OP_W1A8_EX:
       return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double)) +
              align256(size_t(M) * sizeof(LnTokenStats)) + 256;
+    case BL_OP_W1A16_STACK: return kStackMaxLevels * sizeof(uint32_t);
     default: return 0;
   }
 }
@@ -502,6 +535,90 @@ int bitlinear_w1a8_ex(const uint16_t* x, const uint32_t* packed, const float* be
   const unsigned quant = flags & (BL_W1A8_PER_TENSOR | BL_W1A8_NONNEG);
   return w1a8_impl(x, packed, beta, y, M, N, K, ws, ws_bytes, xq_out, gamma_out, acc_out, nullptr, nullptr,
                    (flags & BL_W1A8_TERNARY) != 0, stream, quant);
+}
+
+int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const bl_stack_job* jobs,
+                           int num_jobs, void* ws, size_t ws_bytes, void* stream) {
+  if (num_levels < 0 || num_jobs < 0) return BL_ERR_INVALID_ARG;
+  if (num_levels == 0) return BL_OK;
+  if (!levels || !jobs || !ws || !aligned16(ws) || ws_bytes < bl_workspace_bytes(BL_OP_W1A16_STACK, 0, 0, 0))
+    return BL_ERR_INVALID_ARG;
+  for (int i = 0; i < num_levels; ++i) {
+    const bl_stack_level& lv = levels[i];
+    if (!lv.x || !aligned16(lv.x) || lv.num_jobs < 1 || lv.first_job < 0 ||
+        int64_t(lv.first_job) + lv.num_jobs > num_jobs || lv.num_jobs > kStackMaxJobs)
+      return BL_ERR_INVALID_ARG;
+    if (lv.K < 256 || lv.K > 32 * kStackCluster * 16 * kStackPages || lv.K % 256 != 0) return BL_ERR_UNSUPPORTED;
+    for (int j = lv.first_job; j < lv.first_job + lv.num_jobs; ++j) {
+      const bl_stack_job& jb = jobs[j];
+      if (!jb.packed || !jb.alpha || !jb.y || jb.N < 1) return BL_ERR_INVALID_ARG;
+      if (jb.N > kMaxDim || jb.N * lv.K >= kMaxProduct) return BL_ERR_UNSUPPORTED;
+    }
+  }
+  int sms = 0;
+  int rc = device_setup(&sms);
+  if (rc != BL_OK) return rc;
+  const int G = stack_cluster_capacity();
+  if (G < 1) return BL_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* done = static_cast<uint32_t*>(ws);
+  // one launch per run of at most kStackMaxLevels levels / kStackMaxJobs linears
+  static thread_local StackParams P;  // 12 KB: too large for the stack of every caller
+  int i = 0;
+  while (i < num_levels) {
+    std::memset(&P, 0, sizeof P);
+    int nl = 0, nj = 0;
+    int64_t max_blocks = 0;
+    while (i < num_levels && nl < kStackMaxLevels && nj + levels[i].num_jobs <= kStackMaxJobs) {
+      const bl_stack_level& lv = levels[i];
+      StackLevel& d = P.lv[nl];
+      d.x = lv.x;
+      d.K = int(lv.K);
+      d.job0 = nj;
+      d.njobs = lv.num_jobs;
+      int64_t blocks = 0;
+      for (int j = lv.first_job; j < lv.first_job + lv.num_jobs; ++j) {
+        StackJob& e = P.jb[nj++];
+        e.packed = jobs[j].packed;
+        e.alpha = jobs[j].alpha;
+        e.y = jobs[j].y;
+        e.N = int(jobs[j].N);
+        e.block0 = int(blocks);
+        blocks += cdiv(jobs[j].N, kLutRowsPerCluster);
+      }
+      if (blocks > kMaxDim) return BL_ERR_UNSUPPORTED;
+      d.nblocks = int(blocks);
+      if (blocks > max_blocks) max_blocks = blocks;
+      ++nl;
+      ++i;
+    }
+    const int clusters = int(max_blocks < G ? max_blocks : G);
+    P.done = done;
+    P.num_levels = nl;
+    P.total_ctas = clusters * kStackCluster;
+    if (cudaMemsetAsync(done, 0, size_t(nl) * sizeof(uint32_t), s) != cudaSuccess) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kStackCluster, static_cast<unsigned>(clusters), 1);
+    cfg.blockDim = dim3(kLutThreads, 1, 1);
+    cfg.dynamicSmemBytes = kStackPages * kLutPageBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kStackCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemv_w1a16_stack_kernel, P) != cudaSuccess) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    if ((rc = launch_status()) != BL_OK) return rc;
+  }
+  return BL_OK;
 }
 
 int bitlinear_w158a8_debug(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,

@@ -30,6 +30,8 @@ enum : int {
   kWhereGemmMma = 3,
   kWhereGemmEpilogue = 4,
   kWhereLutInbox = 5,
+  kWhereStackLevel = 6,  // a level waited for the previous one
+  kWhereStackInbox = 7,
 };
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.

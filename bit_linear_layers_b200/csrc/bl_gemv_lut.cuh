@@ -63,6 +63,111 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
                : "memory");
 }
 
+// ---- pieces shared with the multi-layer decode kernel ----
+
+// Packed words of 16 row pairs of one warp (rows w0 + 2p + h), NP pages of
+// this CTA's slice; rows past N and words past the slice read as zero.
+template <int NP>
+__device__ __forceinline__ void lut_load_rows(uint32_t (&wv)[16][NP], const uint32_t* __restrict__ packed,
+                                              int N, int words, int w0, int slice0, int slice_words, int h,
+                                              int wl) {
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    const int row = w0 + 2 * p + h;
+#pragma unroll
+    for (int pg = 0; pg < NP; ++pg) {
+      const int wi = pg * 16 + wl;
+      wv[p][pg] = (row < N && wi < slice_words)
+                      ? __ldcs(packed + static_cast<int64_t>(row) * words + slice0 + wi)
+                      : 0u;
+    }
+  }
+}
+
+// Table of a slice whose first input is xs[0]. Task = (page, value quarter,
+// column); column c holds byte i = c/16 of word c%16. kCoherent reads x
+// through L2 only (it may have been written by other CTAs of the same launch).
+template <int NP, bool kCoherent>
+__device__ __forceinline__ void lut_build_table(const uint16_t* __restrict__ xs, int slice_words,
+                                                uint8_t* lut_smem) {
+  for (int task = threadIdx.x; task < NP * 4 * 64; task += kLutThreads) {
+    const int c = task & 63, qtr = (task >> 6) & 3, pg = task >> 8;
+    const int wi = pg * 16 + (c & 15);
+    if (wi >= slice_words) continue;
+    const int g = 4 * wi + (c >> 4);  // byte position within the slice
+    const uint4* src = reinterpret_cast<const uint4*>(xs + 8 * g);
+    const uint4 raw = kCoherent ? __ldcg(src) : *src;
+    const float x0 = bf16_bits_to_float(raw.x & 0xFFFFu), x1 = __uint_as_float(raw.x & 0xFFFF0000u);
+    const float x2 = bf16_bits_to_float(raw.y & 0xFFFFu), x3 = __uint_as_float(raw.y & 0xFFFF0000u);
+    const float x4 = bf16_bits_to_float(raw.z & 0xFFFFu), x5 = __uint_as_float(raw.z & 0xFFFF0000u);
+    const float x6 = bf16_bits_to_float(raw.w & 0xFFFFu), x7 = __uint_as_float(raw.w & 0xFFFF0000u);
+    // signed pair sums, index = the two bits (bit 0 = lower k)
+    const float p01[4] = {-x0 - x1, x0 - x1, -x0 + x1, x0 + x1};
+    const float p23[4] = {-x2 - x3, x2 - x3, -x2 + x3, x2 + x3};
+    const float p45[4] = {-x4 - x5, x4 - x5, -x4 + x5, x4 + x5};
+    // bits 6 and 7 of this task's values are fixed by its quarter
+    const float q67 = ((qtr & 1) ? x6 : -x6) + ((qtr & 2) ? x7 : -x7);
+    float lo[16];
+#pragma unroll
+    for (int v = 0; v < 16; ++v) lo[v] = p01[v & 3] + p23[v >> 2];
+    float* page = reinterpret_cast<float*>(lut_smem + pg * kLutPageBytes);
+#pragma unroll
+    for (int hq = 0; hq < 4; ++hq) {
+      const int hi = qtr * 4 + hq;
+      const float hv = p45[hq] + q67;
+#pragma unroll
+      for (int v = 0; v < 16; ++v) page[(hi * 16 + v) * 64 + c] = lo[v] + hv;
+    }
+  }
+}
+
+// Lookups of the 16 row pairs over the slice, then a reduce-scatter over the
+// 16 lanes of each half-warp: the return value is the slice's partial sum of
+// row 2 * wl + h of the warp's 32 rows.
+template <int NP>
+__device__ __forceinline__ float lut_row_partial(const uint32_t (&wv)[16][NP], int slice_words,
+                                                 const uint8_t* lut_smem, int h, int wl) {
+  uint32_t sel[4], colb[4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint32_t i = (s + h) & 3;
+    colb[s] = (i * 16 + wl) * 4;
+    sel[s] = 0x5504u | (i << 4);  // byte0 <- column byte, byte1 <- word byte i, bytes 2,3 <- 0
+  }
+  // all 64 lookups of a page are issued before any of them is added, so the
+  // shared-memory latency overlaps (a lane whose word lies past the slice
+  // reads a zero word: its lookups are discarded below)
+  float acc[16];
+#pragma unroll
+  for (int p = 0; p < 16; ++p) acc[p] = 0.f;
+#pragma unroll
+  for (int pg = 0; pg < NP; ++pg) {
+    const uint8_t* page = lut_smem + pg * kLutPageBytes;
+    const bool live = pg * 16 + wl < slice_words;
+    float t[16][4];
+#pragma unroll
+    for (int p = 0; p < 16; ++p)
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        t[p][s] = *reinterpret_cast<const float*>(page + __byte_perm(wv[p][pg], colb[s], sel[s]));
+#pragma unroll
+    for (int p = 0; p < 16; ++p)
+      if (live) acc[p] += (t[p][0] + t[p][1]) + (t[p][2] + t[p][3]);
+  }
+  // reduce-scatter over the 16 lanes of each half: lane wl ends with row pair wl
+#pragma unroll
+  for (int d = 8, n = 16; d >= 1; d >>= 1, n >>= 1) {
+    const bool upper = (wl & d) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = upper ? acc[j] : acc[j + n / 2];
+      const float keep = upper ? acc[j + n / 2] : acc[j];
+      acc[j] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+    }
+  }
+  return acc[0];
+}
+
 // NP = pages (16-word groups) per slice; slice_words <= 16 * NP.
 // One-page slices fit two CTAs per SM (registers capped at 128), which lets
 // an overlapped next launch co-reside with the one finishing.
@@ -91,96 +196,20 @@ __global__ void __launch_bounds__(kLutThreads, NP == 1 ? 2 : 1) gemv_w1a16_lut_k
   cluster_arrive_relaxed();  // waited on just before the first push
 
   // ---- 1. prefetch this warp's packed words (independent of x) ----
-  const int wrow0 = row0 + warp * 32;
   uint32_t wv[16][NP];
-#pragma unroll
-  for (int p = 0; p < 16; ++p) {
-    const int row = wrow0 + 2 * p + h;
-#pragma unroll
-    for (int pg = 0; pg < NP; ++pg) {
-      const int wi = pg * 16 + wl;
-      wv[p][pg] = (row < N && wi < slice_words)
-                      ? __ldcs(packed + static_cast<int64_t>(row) * words + slice0 + wi)
-                      : 0u;
-    }
-  }
+  lut_load_rows<NP>(wv, packed, N, words, row0 + warp * 32, slice0, slice_words, h, wl);
 
   // x may be produced by the previous kernel on the stream
   grid_dependency_wait();
   grid_dependents_launch();
 
   // ---- 2. build the table of this slice ----
-  // task: (page, value quarter, column); column c holds byte i = c/16 of word c%16
-  for (int task = threadIdx.x; task < NP * 4 * 64; task += kLutThreads) {
-    const int c = task & 63, qtr = (task >> 6) & 3, pg = task >> 8;
-    const int wi = pg * 16 + (c & 15);
-    if (wi >= slice_words) continue;
-    const int g = 4 * wi + (c >> 4);  // byte position within the slice
-    const uint4 raw = *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(slice0) * 32 + 8 * g);
-    const float x0 = bf16_bits_to_float(raw.x & 0xFFFFu), x1 = __uint_as_float(raw.x & 0xFFFF0000u);
-    const float x2 = bf16_bits_to_float(raw.y & 0xFFFFu), x3 = __uint_as_float(raw.y & 0xFFFF0000u);
-    const float x4 = bf16_bits_to_float(raw.z & 0xFFFFu), x5 = __uint_as_float(raw.z & 0xFFFF0000u);
-    const float x6 = bf16_bits_to_float(raw.w & 0xFFFFu), x7 = __uint_as_float(raw.w & 0xFFFF0000u);
-    // signed pair sums, index = the two bits (bit 0 = lower k)
-    const float p01[4] = {-x0 - x1, x0 - x1, -x0 + x1, x0 + x1};
-    const float p23[4] = {-x2 - x3, x2 - x3, -x2 + x3, x2 + x3};
-    const float p45[4] = {-x4 - x5, x4 - x5, -x4 + x5, x4 + x5};
-    // bits 6 and 7 of this task's values are fixed by its quarter
-    const float q67 = ((qtr & 1) ? x6 : -x6) + ((qtr & 2) ? x7 : -x7);
-    float lo[16];
-#pragma unroll
-    for (int v = 0; v < 16; ++v) lo[v] = p01[v & 3] + p23[v >> 2];
-    float* page = reinterpret_cast<float*>(lut_smem + pg * kLutPageBytes);
-#pragma unroll
-    for (int hq = 0; hq < 4; ++hq) {
-      const int hi = qtr * 4 + hq;
-      const float hv = p45[hq] + q67;
-#pragma unroll
-      for (int v = 0; v < 16; ++v) page[(hi * 16 + v) * 64 + c] = lo[v] + hv;
-    }
-  }
+  lut_build_table<NP, false>(x + static_cast<int64_t>(slice0) * 32, slice_words, lut_smem);
   __syncthreads();
 
-  // ---- 3. lookups: per row pair, per page, four bytes per lane ----
-  uint32_t sel[4], colb[4];
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const uint32_t i = (s + h) & 3;
-    colb[s] = (i * 16 + wl) * 4;
-    sel[s] = 0x5504u | (i << 4);  // byte0 <- column byte, byte1 <- word byte i, bytes 2,3 <- 0
-  }
-  // all 64 lookups of a page are issued before any of them is added, so the
-  // shared-memory latency overlaps (a lane whose word lies past the slice
-  // reads a zero word: its lookups are discarded below)
-  float acc[16];
-#pragma unroll
-  for (int p = 0; p < 16; ++p) acc[p] = 0.f;
-#pragma unroll
-  for (int pg = 0; pg < NP; ++pg) {
-    const uint8_t* page = lut_smem + pg * kLutPageBytes;
-    const bool live = pg * 16 + wl < slice_words;
-    float t[16][4];
-#pragma unroll
-    for (int p = 0; p < 16; ++p)
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-        t[p][s] = *reinterpret_cast<const float*>(page + __byte_perm(wv[p][pg], colb[s], sel[s]));
-#pragma unroll
-    for (int p = 0; p < 16; ++p)
-      if (live) acc[p] += (t[p][0] + t[p][1]) + (t[p][2] + t[p][3]);
-  }
+  // ---- 3./4. lookups and the per-row reduce-scatter ----
+  const float part = lut_row_partial<NP>(wv, slice_words, lut_smem, h, wl);
 
-  // ---- 4. reduce-scatter over the 16 lanes of each half: lane wl ends with row pair wl ----
-#pragma unroll
-  for (int d = 8, n = 16; d >= 1; d >>= 1, n >>= 1) {
-    const bool upper = (wl & d) != 0;
-#pragma unroll
-    for (int j = 0; j < n / 2; ++j) {
-      const float send = upper ? acc[j] : acc[j + n / 2];
-      const float keep = upper ? acc[j + n / 2] : acc[j];
-      acc[j] = keep + __shfl_xor_sync(0xffffffffu, send, d);
-    }
-  }
   // ---- 5. push each row's partial to its owner; the owner adds the C partials ----
   if (threadIdx.x == 0) mbar_arrive_expect_tx(smem_u32(&inbox_bar), kLutRowsPerCluster * 4);
   cluster_wait();  // every CTA's inbox barrier is initialised
@@ -188,7 +217,7 @@ __global__ void __launch_bounds__(kLutThreads, NP == 1 ? 2 : 1) gemv_w1a16_lut_k
     const int r = warp * 32 + 2 * wl + h;  // this lane's row within the cluster
     const uint32_t owner = static_cast<uint32_t>(r / rows_per_cta);
     const uint32_t slot = smem_u32(&inbox[static_cast<int>(rank) * rows_per_cta + r % rows_per_cta]);
-    st_async_f32(map_to_rank(slot, owner), acc[0], map_to_rank(smem_u32(&inbox_bar), owner));
+    st_async_f32(map_to_rank(slot, owner), part, map_to_rank(smem_u32(&inbox_bar), owner));
   }
   if (threadIdx.x < rows_per_cta) {
     const int r = static_cast<int>(rank) * rows_per_cta + threadIdx.x;

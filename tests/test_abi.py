@@ -87,6 +87,23 @@ def test_null_and_misaligned_pointers_rejected():
     assert bl.lib.bin_pack(FAKE, 128, 96, bl.BL_PACK_FBI, FAKE, FAKE, None, None, 0, None) == -2
 
 
+def test_stack_validation_without_device_work():
+    import bit_linear_layers_b200 as bl
+    job = bl.StackJob(FAKE.value, FAKE.value, FAKE.value, 256)
+    ws = bl.workspace_bytes(bl.BL_OP_W1A16_STACK, 0, 0, 0)
+    assert ws >= 128 * 4
+
+    def call(K, first=0, num=1, n_levels=1, ws_bytes=ws, x=FAKE.value):
+        lv = bl.StackLevel(x, K, first, num)
+        return bl.lib.bin_linear_w1a16_stack(ctypes.byref(lv), n_levels, ctypes.byref(job), 1, FAKE, ws_bytes, None)
+
+    assert call(4096, n_levels=0) == 0              # empty stack: nothing to do
+    assert call(4000) == -2 and call(12544) == -2   # K % 256, more than three table pages
+    assert call(4096, first=1) == -1 and call(4096, num=0) == -1
+    assert call(4096, ws_bytes=8) == -1
+    assert call(4096, x=ODD.value) == -1
+
+
 def test_zero_tokens_is_a_noop():
     import bit_linear_layers_b200 as bl
     assert bl.lib.bin_linear_w1a16(None, FAKE, FAKE, None, 0, 128, 128, None) == 0

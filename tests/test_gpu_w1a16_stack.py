@@ -1,0 +1,172 @@
+"""bin_linear_w1a16_stack (single-token decode through a stack of FBI-linear
+layers in one persistent launch) on the GPU.
+
+* every output of every level against the oracle's W1A16 forward of the
+  input that level actually read (the tolerance of tests/parity.py), for
+  slices of one, two and three table pages, ragged N, several linears per
+  level, and inputs produced by earlier levels;
+* bit-identical to bin_linear_w1a16 called layer by layer where that call
+  also splits K eight ways (K = 4096 and 11008, the 7B shapes);
+* stacks longer than one launch (more than 128 levels or 256 linears);
+* the argument checks."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from parity import bf16_to_f64, check_w1a16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bl():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import bit_linear_layers_b200 as m
+    return m
+
+
+def _linear(oracle, N, K, seed):
+    from bit_linear_layers_b200 import synthetic
+    W = synthetic.weights(N, K, seed)
+    packed, alpha = oracle.pack_fbi(W.numpy())
+    return (torch.from_numpy(packed.view(np.int32)).cuda(), torch.from_numpy(alpha).cuda(), packed, alpha)
+
+
+def _check_level(oracle, x_dev, linears, what):
+    """linears: (packed_np, alpha_np, y_dev) of one level; x_dev the level input."""
+    from bit_linear_layers_b200 import synthetic
+    xb = synthetic.bf16_bits(x_dev.reshape(1, -1))
+    K = xb.shape[1]
+    for i, (packed, alpha, y) in enumerate(linears):
+        y_ref = oracle.w1a16(xb, packed, alpha, K).ravel()
+        N = packed.shape[0]
+        check_w1a16(bf16_to_f64(y.reshape(1, -1)).ravel(), y_ref, alpha, xb, np.zeros(N, np.int64), np.arange(N),
+                    what=f"{what} linear {i}")
+
+
+def _run_and_check(bl, oracle, spec, seed0):
+    """spec: list of levels, each (K, [N...], src) where src is None (a fresh
+    input) or (level, linear) whose output feeds this level."""
+    from bit_linear_layers_b200 import synthetic
+    levels, host, outs = [], [], []
+    for li, (K, Ns, src) in enumerate(spec):
+        if src is None:
+            x = synthetic.activations(1, K, seed0 + 1000 * li).reshape(K).cuda()
+        else:
+            x = outs[src[0]][src[1]]
+            assert x.numel() == K
+        lins, hl, ys = [], [], []
+        for j, N in enumerate(Ns):
+            dp, da, packed, alpha = _linear(oracle, N, K, seed0 + 1000 * li + 7 * j + 1)
+            y = torch.full((N,), float("nan"), dtype=torch.bfloat16, device="cuda")
+            lins.append((dp, da, y))
+            hl.append((packed, alpha, y))
+            ys.append(y)
+        levels.append((x, lins))
+        host.append((x, hl))
+        outs.append(ys)
+    st = bl.W1A16Stack(levels)
+    st.run()
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
+    for li, (x, hl) in enumerate(host):
+        _check_level(oracle, x, hl, f"level {li} (K={spec[li][0]})")
+    return levels, outs
+
+
+def test_stack_one_level_each_page_count(bl, oracle):
+    # slices of 1..48 words: K = 256 (1 word), 3072 (12), 4096 (16), 8192 (32), 11008 (43), 12288 (48)
+    spec = [(256, [100], None), (3072, [256], None), (4096, [300, 1], None), (8192, [513], None),
+            (11008, [1000], None), (12288, [257], None)]
+    _run_and_check(bl, oracle, spec, seed0=3)
+
+
+def test_stack_chained_levels(bl, oracle):
+    # a miniature transformer block stack: x -> (q, k, v); v -> o; o -> (gate, up); up -> down; repeat
+    spec = []
+    for layer in range(3):
+        base = len(spec)
+        src = None if layer == 0 else (base - 1, 0)
+        spec.append((1024, [1024, 1024, 1024], src))   # q, k, v
+        spec.append((1024, [1024], (base, 2)))         # o from v
+        spec.append((1024, [2816, 2816], (base + 1, 0)))  # gate, up from o
+        spec.append((2816, [1024], (base + 2, 1)))     # down from up
+    _run_and_check(bl, oracle, spec, seed0=11)
+
+
+def test_stack_matches_layer_by_layer_at_7b_shapes(bl, oracle):
+    """K = 4096 and 11008 split 8 ways in both calls: identical bits."""
+    from bit_linear_layers_b200 import synthetic
+    shapes = [(4096, 4096), (4096, 4096), (4096, 11008), (11008, 4096)]  # (K, N)
+    x0 = synthetic.activations(1, 4096, 5).reshape(4096).cuda()
+    mats = [_linear(oracle, N, K, 20 + i)[:2] for i, (K, N) in enumerate(shapes)]
+    ys = [torch.empty(N, dtype=torch.bfloat16, device="cuda") for _, N in shapes]
+    levels = [(x0, [(mats[0][0], mats[0][1], ys[0])]), (ys[0], [(mats[1][0], mats[1][1], ys[1])]),
+              (ys[1], [(mats[2][0], mats[2][1], ys[2])]), (ys[2], [(mats[3][0], mats[3][1], ys[3])])]
+    bl.W1A16Stack(levels).run()
+    ref = []
+    cur = x0.reshape(1, -1)
+    for (dp, da), (K, N) in zip(mats, shapes):
+        cur = bl.bin_linear_w1a16(cur, dp, da)
+        ref.append(cur.reshape(N))
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(zip(ys, ref)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"level {i} differs"
+
+
+def test_stack_longer_than_one_launch(bl, oracle):
+    # 140 levels (two launches), alternating between two buffers
+    from bit_linear_layers_b200 import synthetic
+    K = N = 512
+    dp, da, packed, alpha = _linear(oracle, N, K, 77)
+    x0 = synthetic.activations(1, K, 78).reshape(K).cuda()
+    bufs = [torch.empty(K, dtype=torch.bfloat16, device="cuda") for _ in range(140)]
+    levels = [(x0 if i == 0 else bufs[i - 1], [(dp, da, bufs[i])]) for i in range(140)]
+    bl.W1A16Stack(levels).run()
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
+    for i in (0, 1, 127, 128, 129, 139):
+        x = x0 if i == 0 else bufs[i - 1]
+        _check_level(oracle, x, [(packed, alpha, bufs[i])], f"level {i}")
+
+
+def test_stack_many_linears_per_launch(bl, oracle):
+    # 300 linears over 3 levels (more than 256 linears: split between launches)
+    from bit_linear_layers_b200 import synthetic
+    K = 256
+    dp, da, packed, alpha = _linear(oracle, 64, K, 90)
+    xs = [synthetic.activations(1, K, 91 + i).reshape(K).cuda() for i in range(3)]
+    ys = [[torch.empty(64, dtype=torch.bfloat16, device="cuda") for _ in range(100)] for _ in range(3)]
+    levels = [(xs[i], [(dp, da, y) for y in ys[i]]) for i in range(3)]
+    bl.W1A16Stack(levels).run()
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
+    for i in range(3):
+        _check_level(oracle, xs[i], [(packed, alpha, y) for y in ys[i][::33]], f"level {i}")
+
+
+def test_stack_argument_checks(bl):
+    K, N = 4096, 256
+    x = torch.zeros(K, dtype=torch.bfloat16, device="cuda")
+    p = torch.zeros((N, K // 32), dtype=torch.int32, device="cuda")
+    a = torch.zeros(N, dtype=torch.float32, device="cuda")
+    y = torch.zeros(N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(bl.workspace_bytes(bl.BL_OP_W1A16_STACK, 0, 0, 0), dtype=torch.uint8, device="cuda")
+    job = bl.StackJob(p.data_ptr(), a.data_ptr(), y.data_ptr(), N)
+
+    def call(K_, first=0, num=1, ws_bytes=ws.numel(), xp=x.data_ptr()):
+        lv = bl.StackLevel(xp, K_, first, num)
+        return bl.lib.bin_linear_w1a16_stack(ctypes.byref(lv), 1, ctypes.byref(job), 1, ws.data_ptr(), ws_bytes,
+                                             torch.cuda.current_stream().cuda_stream)
+
+    assert call(4096) == 0
+    assert call(4000) == bl.BL_ERR_UNSUPPORTED     # not a multiple of 256
+    assert call(12544) == bl.BL_ERR_UNSUPPORTED    # beyond three table pages
+    assert call(4096, first=1) == bl.BL_ERR_INVALID_ARG
+    assert call(4096, num=0) == bl.BL_ERR_INVALID_ARG
+    assert call(4096, ws_bytes=4) == bl.BL_ERR_INVALID_ARG
+    assert call(4096, xp=x.data_ptr() + 2) == bl.BL_ERR_INVALID_ARG  # x not 16-byte aligned
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
