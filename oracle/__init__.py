@@ -48,6 +48,7 @@ class Oracle:
             "oracle_ln_quant_tensor": [_p, _i64, _i64, _dbl, ctypes.c_int, _p, _p, _p, _p],
             "oracle_w158a8_acc": [_p, _p, _i64, _i64, _i64, _p],
             "oracle_w158a8_acc_at": [_p, _p, _i64, _p, _p, _i64, _p],
+            "oracle_w1a16_backward": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -89,6 +90,23 @@ class Oracle:
         y = np.zeros((M, N), dtype=np.float64)
         self._lib.oracle_w1a16(_ptr(x), _ptr(packed), _ptr(alpha), M, N, K, _ptr(y))
         return y
+
+    def w1a16_backward(self, x_bf16: np.ndarray, packed: np.ndarray, alpha: np.ndarray, dy_bf16: np.ndarray,
+                       K: int):
+        """FBI-linear backward with the straight-through estimator (reading
+        R18): returns (dx [M, K], dw [N, K], dalpha [N]) in fp64."""
+        x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+        dy = np.ascontiguousarray(dy_bf16, dtype=np.uint16)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+        M, N = dy.shape
+        assert x.shape == (M, K) and packed.shape == (N, self.row_words(K)) and alpha.shape == (N,)
+        dx = np.zeros((M, K), dtype=np.float64)
+        dw = np.zeros((N, K), dtype=np.float64)
+        da = np.zeros(N, dtype=np.float64)
+        self._lib.oracle_w1a16_backward(_ptr(x), _ptr(packed), _ptr(alpha), _ptr(dy), M, N, K, _ptr(dx), _ptr(dw),
+                                        _ptr(da))
+        return dx, dw, da
 
     def w1a16_at(self, x_bf16, packed, alpha, K: int, ms, js):
         x = np.ascontiguousarray(x_bf16, dtype=np.uint16)

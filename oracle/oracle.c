@@ -42,25 +42,34 @@
  *       element (j,k) is bit (k mod 32) of word [j*ceil(K/32) + k/32]; a set
  *       bit means +1, a clear bit -1; unused bits of a row's last word are 0.
  *   R9  Activations are bf16 (raw 16-bit patterns in, decoded exactly).
- *   R10 b1.58 weights ([BitNet] section 2, Eq.(9)-(11)): the epsilon of
+ *   R11 b1.58 weights ([BitNet] section 2, Eq.(9)-(11)): the epsilon of
  *       Eq.(9) is not given; it is a parameter (the library uses 1e-5).
- *   R11 "round" in Eq.(10): to nearest, ties to even (as R5), applied to
+ *   R12 "round" in Eq.(10): to nearest, ties to even (as R5), applied to
  *       W / (gamma + eps) evaluated in fp64.
- *   R12 Packed ternary layout (the library's written spec): row j takes
+ *   R13 Packed ternary layout (the library's written spec): row j takes
  *       ceil(K/128) blocks of 8 uint32 words; block b covers k in
  *       [128b, 128b + 128): its words 0-3 are the +1 plane, words 4-7 the
  *       -1 plane, element k at bit (k mod 32) of word (k mod 128)/32 of each
  *       plane. A weight is +1, -1 or 0 (neither bit set); never both.
- *   R14 Per-tensor activation scale ([BitNet] Eq.(5) literally: "of the input
+ *   R15 Per-tensor activation scale ([BitNet] Eq.(5) literally: "of the input
  *       matrix"): gamma = max |LN(x)| over all M x K elements, shared by all
  *       tokens; codes as R5.
- *   R15 Eq.(6) (activations before a nonlinearity): eta = min over all M x K
+ *   R16 Eq.(6) (activations before a nonlinearity): eta = min over all M x K
  *       LN values, gamma = max over all of (LN - eta), so (LN - eta) * Q_b /
  *       gamma lies in [0, Q_b]; rounded to nearest (ties to even) and clamped
- *       to [0, 127] (the clip bounds eps and Q_b - eps as integers). The
- *       forward then applies Eq.(7) as printed, y = acc * beta * gamma / Q_b
+ *       to [0, 127] (the clip bounds eps and Q_b - eps as integers).
+ *   R17 The forward then applies Eq.(7) as printed, y = acc * beta * gamma / Q_b
  *       (the pages give no term for eta). gamma == 0 gives all-zero codes.
- *   R13 The b1.58 forward is the BitLinear forward of Eq.(7) with the
+ *   R18 FBI-linear backward ([FBI]: the straight-through estimator carries
+ *       the gradient through the sign function). With y_mj = alpha_j * z_mj,
+ *       z_mj = sum_k s_jk x_mk and an incoming gradient dy (M x N):
+ *         dx_mk    = sum_j dy_mj * alpha_j * s_jk        (exact chain rule)
+ *         dalpha_j = sum_m dy_mj * z_mj                 (exact chain rule)
+ *         dW_jk    = alpha_j * sum_m dy_mj * x_mk        (STE: ds/dW taken as 1)
+ *       The page names the estimator but gives no clipping window, so the
+ *       plain identity form is used (no |W| <= 1 gate); dW is the gradient of
+ *       the latent full-precision weight. dy is bf16 like the activations.
+ *   R14 The b1.58 forward is the BitLinear forward of Eq.(7) with the
  *       ternary weights: the same LN and activation quantisation (section 2
  *       keeps BitNet's), and the rescale uses gamma of Eq.(11) as beta (Eq.(11)
  *       and the beta of Eq.(8) are the same mean of |W|).
@@ -225,7 +234,7 @@ void oracle_ln_absmax_quant(const uint16_t* x, int64_t M, int64_t K, double eps,
     }
 }
 
-/* Per-tensor variants of the activation quantisation, readings R14 and R15,
+/* Per-tensor variants of the activation quantisation, readings R15 and R16,
  * on the LN output of every token (LN as in oracle_ln_absmax_quant):
  *   mode 0 (Eq.(5), per tensor):  gamma = max_{m,k} |LN_mk|
  *          q_mk = clamp(rne(LN_mk * Q_b / gamma), -127, 127)
@@ -322,7 +331,7 @@ void oracle_w1a8_rescale(const int64_t* acc, const double* gamma, double beta,
 
 static int64_t ternary_row_words(int64_t K) { return ((K + 127) / 128) * 8; }
 
-/* read element (j,k) of a packed ternary matrix as +1 / 0 / -1 (layout R12) */
+/* read element (j,k) of a packed ternary matrix as +1 / 0 / -1 (layout R13) */
 static int ternary_value(const uint32_t* packed, int64_t K, int64_t j, int64_t k)
 {
     const uint32_t* blk = packed + j * ternary_row_words(K) + (k / 128) * 8;
@@ -332,7 +341,7 @@ static int ternary_value(const uint32_t* packed, int64_t K, int64_t j, int64_t k
     return (int)plus - (int)minus;
 }
 
-/* [BitNet] section 2, Eq.(9)-(11), readings R10-R12:
+/* [BitNet] section 2, Eq.(9)-(11), readings R11-R13:
  *   gamma  = (1/(N K)) * sum_jk |W_jk|                      (fp64)
  *   W~_jk  = RoundClip(W_jk / (gamma + eps), -1, 1)
  *          = max(-1, min(1, round_half_even(W_jk / (gamma + eps))))  */
@@ -357,7 +366,7 @@ void oracle_pack_ternary(const float* W, int64_t N, int64_t K, double eps, uint3
     *gamma_out = gamma;
 }
 
-/* integer core of Eq.(7) with ternary weights (R13):
+/* integer core of Eq.(7) with ternary weights (R14):
  *   acc_mj = sum_k W~_jk * q_mk          (int64) */
 static int64_t w158a8_acc_one(const int8_t* xq, const uint32_t* packed, int64_t K,
                               int64_t m, int64_t j)
@@ -381,6 +390,43 @@ void oracle_w158a8_acc_at(const int8_t* xq, const uint32_t* packed, int64_t K,
 {
     for (int64_t i = 0; i < count; ++i)
         acc[i] = w158a8_acc_one(xq, packed, K, ms[i], js[i]);
+}
+
+/* ---- FBI-linear backward with the straight-through estimator ----------- */
+
+/* [FBI] training paragraph and reading R18. x (M x K) and dy (M x N) are
+ * bf16 patterns, packed the N x K signs (R8), alpha the N scales. Outputs in
+ * fp64: dx (M x K), dw (N x K), dalpha (N). Each is its definition summed in
+ * the obvious order; z (the forward's unscaled products) is formed first
+ * because dalpha is defined through it. */
+void oracle_w1a16_backward(const uint16_t* x, const uint32_t* packed, const float* alpha,
+                           const uint16_t* dy, int64_t M, int64_t N, int64_t K,
+                           double* dx, double* dw, double* dalpha)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t j = 0; j < N; ++j)
+                s += bf16_value(dy[m * N + j]) * (double)alpha[j] * (double)packed_sign(packed, K, j, k);
+            dx[m * K + k] = s;
+        }
+    for (int64_t j = 0; j < N; ++j)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t m = 0; m < M; ++m)
+                s += bf16_value(dy[m * N + j]) * bf16_value(x[m * K + k]);
+            dw[j * K + k] = (double)alpha[j] * s;
+        }
+    for (int64_t j = 0; j < N; ++j) {
+        double s = 0.0;
+        for (int64_t m = 0; m < M; ++m) {
+            double z = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                z += (double)packed_sign(packed, K, j, k) * bf16_value(x[m * K + k]);
+            s += bf16_value(dy[m * N + j]) * z;
+        }
+        dalpha[j] = s;
+    }
 }
 
 /* ---- W1A1 (only as an identity check of the packed-sign reading) ------- */

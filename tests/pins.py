@@ -20,7 +20,10 @@ What pins what:
   tokens, exact .5 ties (round half to even);
 * for the b1.58 ternary weights: a hand-worked example with exact ties and
   clips, equal-magnitude weights reducing to the binary signs (through the
-  separate FBI packing), popcount closed forms, inert sub-threshold weights.
+  separate FBI packing), popcount closed forms, inert sub-threshold weights;
+* for the straight-through backward: adjoint identities against the
+  forward, exact unit-step differences of the forward, all-ones closed
+  forms, and dw's independence of the signs (with numpy's matmul).
 """
 from __future__ import annotations
 
@@ -449,6 +452,95 @@ def pin_quant_nonneg_range(o):
     i_min, i_max = np.unravel_index(np.argmin(pre), pre.shape), np.unravel_index(np.argmax(pre), pre.shape)
     assert xq[i_min] == 0 and xq[i_max] == 127 and pre[i_min] == 0.0 and pre[i_max] == 128.0
     assert eta < 0 < gamma[0] and np.all(gamma == gamma[0])
+
+
+# ---------------------------------------------------------------- backward (STE)
+#
+# The forward is linear in x and in alpha, so its gradients are fixed by the
+# forward alone: <dy, y> = <dx, x> = <dalpha, alpha> (adjoint identities), a
+# unit step in x_mk or alpha_j changes <dy, y> by exactly dx_mk or dalpha_j,
+# and the straight-through weight gradient satisfies <dw, S> = <dy, y> too
+# (dw_jk = alpha_j sum_m dy_mj x_mk, summed against s_jk gives alpha_j z_mj).
+
+
+def _backward_case(seed, M, N, K, small_ints=False):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    if small_ints:  # values whose unit steps stay exact in bf16
+        x = _bf16_bits_of(rng.integers(-8, 9, M * K).tolist()).reshape(M, K)
+        dy = _bf16_bits_of(rng.integers(-4, 5, M * N).tolist()).reshape(M, N)
+    else:
+        x = _to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+        dy = _to_bf16_bits(rng.standard_normal((M, N)).astype(np.float32))
+    return W, x, dy
+
+
+def _inner(a, b) -> float:
+    return math.fsum((np.asarray(a, dtype=np.float64) * np.asarray(b, dtype=np.float64)).ravel().tolist())
+
+
+def pin_backward_adjoint_identities(o):
+    M, N, K = 3, 5, 70  # N != K and M != N: a transposed index changes shapes or values
+    W, x, dy = _backward_case(41, M, N, K)
+    packed, alpha = o.pack_fbi(W)
+    y = o.w1a16(x, packed, alpha, K)
+    dx, dw, da = o.w1a16_backward(x, packed, alpha, dy, K)
+    assert dx.shape == (M, K) and dw.shape == (N, K) and da.shape == (N,)
+    ref = _inner(_bf16_values(dy), y)
+    S = np.where(W > 0, 1.0, -1.0)
+    for name, val in (("<dx,x>", _inner(dx, _bf16_values(x))), ("<dalpha,alpha>", _inner(da, alpha)),
+                      ("<dw,S>", _inner(dw, S))):
+        assert abs(val - ref) <= 1e-12 * max(1.0, abs(ref)), (name, val, ref)
+
+
+def pin_backward_unit_steps(o):
+    # small integers: every sum below is exact in fp64, so the differences are exact
+    M, N, K = 2, 3, 40
+    W, x, dy = _backward_case(43, M, N, K, small_ints=True)
+    packed, alpha = o.pack_fbi(W)
+    alpha = np.array([0.5, 2.0, -1.25], dtype=np.float32)  # any scales (exact binary fractions)
+    dyv = _bf16_values(dy)
+    base = _inner(dyv, o.w1a16(x, packed, alpha, K))
+    dx, dw, da = o.w1a16_backward(x, packed, alpha, dy, K)
+    for (m, k) in ((0, 0), (1, 17), (0, 39)):
+        xs = x.copy()
+        xs[m, k] = _bf16_bits_of([_bf16_values(x[m:m + 1, k:k + 1])[0, 0] + 1.0])[0]
+        step = _inner(dyv, o.w1a16(xs, packed, alpha, K)) - base
+        assert step == dx[m, k], ((m, k), step, dx[m, k])
+    for j in range(N):
+        a2 = alpha.copy()
+        a2[j] += np.float32(1.0)
+        step = _inner(dyv, o.w1a16(x, packed, a2, K)) - base
+        assert step == da[j], (j, step, da[j])
+
+
+def pin_backward_all_ones_closed_form(o):
+    M, N, K = 4, 6, 96
+    W, _, _ = _backward_case(47, M, N, K)
+    packed, alpha = o.pack_fbi(W)
+    ones_x = _bf16_bits_of([1] * (M * K)).reshape(M, K)
+    ones_dy = _bf16_bits_of([1] * (M * N)).reshape(M, N)
+    dx, dw, da = o.w1a16_backward(ones_x, packed, alpha, ones_dy, K)
+    S = np.where(W > 0, 1.0, -1.0)
+    # dw_jk = alpha_j * M; dx_mk = sum_j alpha_j s_jk; dalpha_j = M (#pos_j - #neg_j)
+    assert np.array_equal(dw, np.repeat(alpha.astype(np.float64)[:, None] * M, K, axis=1))
+    for k in range(K):
+        want = math.fsum((alpha.astype(np.float64) * S[:, k]).tolist())
+        assert abs(dx[0, k] - want) <= 1e-15 * N and np.all(dx[:, k] == dx[0, k]), k
+    assert np.array_equal(da, M * (2.0 * _popcounts(packed) - K))
+
+
+def pin_backward_dw_ignores_signs(o):
+    # straight-through: dw does not depend on which way the weights' signs went
+    M, N, K = 3, 4, 64
+    W, x, dy = _backward_case(53, M, N, K)
+    packed, alpha = o.pack_fbi(W)
+    _, dw1, _ = o.w1a16_backward(x, packed, alpha, dy, K)
+    _, dw2, _ = o.w1a16_backward(x, packed ^ np.uint32(0xFFFFFFFF), alpha, dy, K)
+    assert np.array_equal(dw1, dw2)
+    # and it is alpha_j times a product that numpy computes independently
+    P = _bf16_values(dy).T @ _bf16_values(x)
+    assert np.allclose(dw1, alpha.astype(np.float64)[:, None] * P, rtol=1e-13, atol=1e-13)
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -76,6 +76,20 @@ MUTANTS = [
     ("ternary_acc_sign_ignored",
      "acc += (int64_t)ternary_value(packed, K, j, k) * (int64_t)xq[m * K + k];",
      "acc += (int64_t)(ternary_value(packed, K, j, k) != 0) * (int64_t)xq[m * K + k];"),
+    # straight-through backward
+    ("backward_dx_without_alpha", "s += bf16_value(dy[m * N + j]) * (double)alpha[j] * (double)packed_sign(packed, K, j, k);",
+     "s += bf16_value(dy[m * N + j]) * (double)packed_sign(packed, K, j, k);"),
+    ("backward_dx_sign_dropped", "s += bf16_value(dy[m * N + j]) * (double)alpha[j] * (double)packed_sign(packed, K, j, k);",
+     "s += bf16_value(dy[m * N + j]) * (double)alpha[j];"),
+    ("backward_dw_without_alpha", "dw[j * K + k] = (double)alpha[j] * s;", "dw[j * K + k] = s;"),
+    ("backward_dw_gated_by_sign", "dw[j * K + k] = (double)alpha[j] * s;",
+     "dw[j * K + k] = (double)alpha[j] * s * (packed_sign(packed, K, j, k) > 0 ? 1.0 : 0.0);"),
+    ("backward_dw_token_row_swapped", "s += bf16_value(dy[m * N + j]) * bf16_value(x[m * K + k]);",
+     "s += bf16_value(dy[m * N + j]) * bf16_value(x[(M - 1 - m) * K + k]);"),
+    ("backward_dalpha_scaled", "        dalpha[j] = s;", "        dalpha[j] = (double)alpha[j] * s;"),
+    ("backward_dalpha_last_input_dropped",
+     "            for (int64_t k = 0; k < K; ++k)\n                z +=",
+     "            for (int64_t k = 0; k < K - 1; ++k)\n                z +="),
 ]
 
 
