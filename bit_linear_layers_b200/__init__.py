@@ -44,6 +44,7 @@ BL_OP_PACK_TERNARY = 4
 BL_OP_W158A8 = 5
 BL_OP_W1A8_EX = 6
 BL_OP_W1A16_STACK = 7
+BL_OP_W1A16_BACKWARD = 8
 
 BL_W1A8_TERNARY = 1
 BL_W1A8_PER_TENSOR = 2
@@ -79,6 +80,7 @@ SIGNATURES = {
     "bitlinear_w1a8_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
     "bin_xnor_gemm": ([_p, _p, _p, _i64, _i64, _i64, _p], _int),
     "bin_linear_w1a16_stack": ([_p, _int, _p, _int, _p, _sz, _p], _int),
+    "bin_linear_w1a16_backward": ([_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w1a8_ex": ([_p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_uint, _p, _sz, _p, _p, _p, _p], _int),
     "bitlinear_w158a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w158a8_debug": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p, _p, _p, _p, _p, _p], _int),
@@ -192,6 +194,34 @@ def bin_linear_w1a16(x: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor,
         rc = lib.bin_linear_w1a16(*args, _stream(x.device))
         _check("bin_linear_w1a16", rc)
     return out
+
+
+def bin_linear_w1a16_backward(x: torch.Tensor, packed: torch.Tensor, alpha: torch.Tensor, dy: torch.Tensor, *,
+                              want_dx: bool = True, want_dw: bool = True, dx=None, dw=None, dalpha=None, ws=None):
+    """Straight-through backward of the FBI-linear forward: returns (dx [M, K]
+    bf16 or None, dw [N, K] fp32 or None, dalpha [N] fp32 or None)."""
+    M, K = x.shape
+    N = packed.shape[0]
+    dev = x.device
+    if want_dx and dx is None:
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    if want_dw and dw is None:
+        dw = torch.empty((N, K), dtype=torch.float32, device=dev)
+    if want_dw and dalpha is None:
+        dalpha = torch.empty(N, dtype=torch.float32, device=dev)
+    if not want_dx:
+        dx = None
+    if not want_dw:
+        dw = dalpha = None
+    ws, _ = _workspace(BL_OP_W1A16_BACKWARD, M, N, K, dev, ws)
+    rc = lib.bin_linear_w1a16_backward(
+        _dev_ptr(x, torch.bfloat16, "x"), _dev_ptr(packed, torch.int32, "packed"),
+        _dev_ptr(alpha, torch.float32, "alpha"), _dev_ptr(dy, torch.bfloat16, "dy"),
+        _dev_ptr(dx, torch.bfloat16, "dx"), _dev_ptr(dw, torch.float32, "dw"),
+        _dev_ptr(dalpha, torch.float32, "dalpha"), M, N, K, _dev_ptr(ws, torch.uint8, "ws"),
+        ws.numel() if ws is not None else 0, _stream(dev))
+    _check("bin_linear_w1a16_backward", rc)
+    return dx, dw, dalpha
 
 
 class W1A16Stack:

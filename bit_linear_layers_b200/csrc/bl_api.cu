@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "bitlinear.h"
+#include "bl_backward.cuh"
 #include "bl_common.cuh"
 #include "bl_gemm_ts.cuh"
 #include "bl_gemv.cuh"
@@ -84,7 +85,8 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<2>, 2 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
               set_ts_smem<0>() && set_ts_smem<1>() && set_ts_smem<2>() &&
-              set_smem(gemv_w1a16_stack_kernel, kStackPages * kLutPageBytes);
+              set_smem(gemv_w1a16_stack_kernel, kStackPages * kLutPageBytes) &&
+              set_smem(gemm_ss_ste_kernel, kSsSmemBytes);
     if (!ok) cudaGetLastError();
     {
       cudaLaunchConfig_t cfg = {};
@@ -430,6 +432,11 @@ size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
       return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double)) +
              align256(size_t(M) * sizeof(LnTokenStats)) + 256;
     case BL_OP_W1A16_STACK: return kStackMaxLevels * sizeof(uint32_t);
+    case BL_OP_W1A16_BACKWARD: {
+      const size_t Mp = size_t(cdiv(M, kSsUnit) * kSsUnit);
+      return align256(size_t(M) * size_t(N) * 4) + align256(size_t(K) * size_t(N) / 4) +
+             align256(size_t(K) * 4) + align256(size_t(K) * Mp * 2) + align256(size_t(N) * Mp * 2);
+    }
     default: return 0;
   }
 }
@@ -616,6 +623,80 @@ int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const b
       cudaGetLastError();
       return BL_ERR_CUDA;
     }
+    if ((rc = launch_status()) != BL_OK) return rc;
+  }
+  return BL_OK;
+}
+
+int bin_linear_w1a16_backward(const uint16_t* x, const uint32_t* packed, const float* alpha, const uint16_t* dy,
+                              uint16_t* dx, float* dw, float* dalpha, int64_t M, int64_t N, int64_t K, void* ws,
+                              size_t ws_bytes, void* stream) {
+  int rc = check_shape(M, N, K);
+  if (rc != BL_OK) return rc;
+  if (N % 128 != 0) return BL_ERR_UNSUPPORTED;
+  if ((dw == nullptr) != (dalpha == nullptr)) return BL_ERR_INVALID_ARG;
+  if (!packed || !alpha || !aligned16(packed) || (dw && !aligned16(dw)) || (dx && !aligned16(dx)))
+    return BL_ERR_INVALID_ARG;
+  const int64_t Mp = cdiv(M, kSsUnit) * kSsUnit;
+  if (cdiv(Mp, 32) > 65535 || cdiv(N, 32) > 65535 || cdiv(K, 32) > 65535) return BL_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 0) {  // an empty batch: zero weight and scale gradients, no dx
+    if (dw && (cudaMemsetAsync(dw, 0, size_t(N) * size_t(K) * 4, s) != cudaSuccess ||
+               cudaMemsetAsync(dalpha, 0, size_t(N) * 4, s) != cudaSuccess)) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    return BL_OK;
+  }
+  if (!x || !dy || !aligned16(x) || !aligned16(dy)) return BL_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < bl_workspace_bytes(BL_OP_W1A16_BACKWARD, M, N, K))
+    return BL_ERR_INVALID_ARG;
+  int sms = 0;
+  rc = device_setup(&sms);
+  if (rc != BL_OK) return rc;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  auto* g2 = reinterpret_cast<uint16_t*>(w);
+  w += align256(size_t(M) * size_t(N) * 4);
+  auto* packed_t2 = reinterpret_cast<uint32_t*>(w);
+  w += align256(size_t(K) * size_t(N) / 4);
+  auto* ones = reinterpret_cast<float*>(w);
+  w += align256(size_t(K) * 4);
+  auto* xt = reinterpret_cast<uint16_t*>(w);
+  w += align256(size_t(K) * size_t(Mp) * 2);
+  auto* dyt = reinterpret_cast<uint16_t*>(w);
+  const unsigned ew_grid = static_cast<unsigned>(sms * 8);
+  if (dx) {
+    // dx = [hi | lo] x [S^T | S^T] through the forward path (unit scales)
+    ste_scale_split_kernel<<<ew_grid, 256, 0, s>>>(dy, alpha, M, N, g2);
+    if ((rc = launch_status()) != BL_OK) return rc;
+    const int64_t warps = (N / 32) * (K / 32);
+    const int64_t blocks = cdiv(warps, 8) < int64_t(sms) * 16 ? cdiv(warps, 8) : int64_t(sms) * 16;
+    transpose_pack_dup_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(packed, N, K, packed_t2);
+    if ((rc = launch_status()) != BL_OK) return rc;
+    fill_f32_kernel<<<static_cast<unsigned>(cdiv(K, 256) < sms ? cdiv(K, 256) : sms), 256, 0, s>>>(ones, K, 1.0f);
+    if ((rc = launch_status()) != BL_OK) return rc;
+    rc = bin_linear_w1a16_ex(g2, packed_t2, ones, dx, M, K, 2 * N, 0u, stream);
+    if (rc != BL_OK) return rc;
+  }
+  if (dw) {
+    // P = dY^T X on the tensor cores, then dW = alpha P and dalpha = sum_k s P in place
+    const dim3 tb(32, 8);
+    transpose_bf16_kernel<<<dim3(unsigned(cdiv(K, 32)), unsigned(cdiv(Mp, 32))), tb, 0, s>>>(x, M, K, xt, Mp);
+    if ((rc = launch_status()) != BL_OK) return rc;
+    transpose_bf16_kernel<<<dim3(unsigned(cdiv(N, 32)), unsigned(cdiv(Mp, 32))), tb, 0, s>>>(dy, M, N, dyt, Mp);
+    if ((rc = launch_status()) != BL_OK) return rc;
+    CUtensorMap tm_a, tm_b;
+    if (!make_map_2d(&tm_a, xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(Mp), uint64_t(K), kSsUnit, kSsRowsA,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tm_b, dyt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(Mp), uint64_t(N), kSsUnit, kSsRowsB,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return BL_ERR_CUDA;
+    const int64_t tiles = (K / kSsRowsA) * cdiv(N, kSsRowsB);
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+    gemm_ss_ste_kernel<<<grid, kSsThreads, kSsSmemBytes, s>>>(tm_a, tm_b, int(K), int(N), int(Mp), dw);
+    if ((rc = launch_status()) != BL_OK) return rc;
+    const int64_t fblocks = cdiv(N, 8) < int64_t(sms) * 16 ? cdiv(N, 8) : int64_t(sms) * 16;
+    ste_finalize_kernel<<<static_cast<unsigned>(fblocks), 256, 0, s>>>(dw, packed, alpha, N, K, dalpha);
     if ((rc = launch_status()) != BL_OK) return rc;
   }
   return BL_OK;

@@ -1,0 +1,261 @@
+// FBI-linear backward with the straight-through estimator ("FBI-LLM" page,
+// FBI-linear paragraph and its training sentence: the estimator carries the
+// gradient through the sign function). With y = alpha_j * z_mj,
+// z_mj = sum_k s_jk x_mk, and the incoming gradient dy (M x N):
+//
+//   dx_mk    = sum_j (dy_mj alpha_j) s_jk      a binarized product: the
+//              forward kernels with the transposed signs (below)
+//   P_jk     = sum_m dy_mj x_mk                 a dense bf16 product (tensor cores)
+//   dW_jk    = alpha_j P_jk                     straight-through: ds/dW = 1
+//   dalpha_j = sum_m dy_mj z_mj = sum_k s_jk P_jk
+//
+// dx runs through the forward path unchanged: with g = dy * alpha split into
+// two bf16 parts g = hi + lo (exact to ~2^-17 of g), dx = [hi | lo] x [S^T | S^T]
+// is a W1A16 product of M tokens, 2N inputs and K outputs with unit scales;
+// transpose_pack_dup_kernel writes S^T (each row twice) in the packed layout.
+// P is a plain tcgen05 GEMM with both operands in shared memory (TMA,
+// 128-byte swizzle), computed as D[k][j] = sum_m X^T[k][m] dY^T[j][m] so that
+// each warp's stores of a column j are contiguous in P's row j.
+#pragma once
+
+#include "bl_common.cuh"
+
+namespace bl {
+
+// ---- element-wise and layout kernels -----------------------------------------------
+
+// g = dy * alpha_j in fp32, split into bf16 hi (round to nearest) and bf16 lo
+// = the rounding of the remainder: row m of g2 is [hi_m0..hi_mN-1 | lo_m0..lo_mN-1]
+__global__ void ste_scale_split_kernel(const uint16_t* __restrict__ dy, const float* __restrict__ alpha, int64_t M,
+                                       int64_t N, uint16_t* __restrict__ g2) {
+  const int64_t total = M * N;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / N, j = i - m * N;
+    const float g = bf16_bits_to_float(dy[i]) * alpha[j];
+    const uint16_t hi = float_to_bf16_bits(g);
+    const uint16_t lo = float_to_bf16_bits(g - bf16_bits_to_float(hi));
+    g2[m * 2 * N + j] = hi;
+    g2[m * 2 * N + N + j] = lo;
+  }
+}
+
+// Packed signs [N][K/32] -> their transpose [K][2N/32], each row written
+// twice (words 0..N/32-1 and again N/32..2N/32-1). One warp per 32 x 32 bit
+// block: lane l holds word (row j0 + l, column word kw); the ballot of bit b
+// over the lanes is word j0/32 of transposed row 32 kw + b. N % 32 == 0.
+__global__ void transpose_pack_dup_kernel(const uint32_t* __restrict__ packed, int64_t N, int64_t K,
+                                          uint32_t* __restrict__ out) {
+  const int64_t nw = N / 32, kw_count = K / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; wid < nw * kw_count;
+       wid += warps) {
+    const int64_t jb = wid / kw_count, kw = wid - jb * kw_count;
+    const uint32_t w = packed[(jb * 32 + lane) * kw_count + kw];
+    uint32_t mine = 0u;
+#pragma unroll
+    for (int b = 0; b < 32; ++b) {
+      const uint32_t col = __ballot_sync(0xffffffffu, (w >> b) & 1u);
+      if (lane == b) mine = col;
+    }
+    uint32_t* row = out + (kw * 32 + lane) * 2 * nw;
+    row[jb] = mine;
+    row[nw + jb] = mine;
+  }
+}
+
+// bf16 [R][C] -> [C][Rp] (Rp >= R; entries r >= R are zero): 32 x 32 tiles
+// through shared memory, block (32, 8)
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int64_t R, int64_t C,
+                                      uint16_t* __restrict__ out, int64_t Rp) {
+  __shared__ uint16_t tile[32][33];
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 32, r0 = static_cast<int64_t>(blockIdx.y) * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    const int64_t r = r0 + ty + i, c = c0 + tx;
+    tile[ty + i][tx] = (r < R && c < C) ? in[r * C + c] : static_cast<uint16_t>(0);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    const int64_t c = c0 + ty + i, r = r0 + tx;
+    if (c < C && r < Rp) out[c * Rp + r] = tile[tx][ty + i];
+  }
+}
+
+__global__ void fill_f32_kernel(float* __restrict__ p, int64_t n, float v) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = v;
+}
+
+// In place over P [N][K] (fp32): dW_jk = alpha_j P_jk, and dalpha_j =
+// sum_k s_jk P_jk (fp64 sum in a fixed order). One warp per row.
+__global__ void ste_finalize_kernel(float* __restrict__ pw, const uint32_t* __restrict__ packed,
+                                    const float* __restrict__ alpha, int64_t N, int64_t K,
+                                    float* __restrict__ dalpha) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t kw_count = K / 32;
+  for (int64_t j = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; j < N; j += warps) {
+    const float a = alpha[j];
+    float* row = pw + j * K;
+    const uint32_t* bits = packed + j * kw_count;
+    double s = 0.0;
+    for (int64_t kw = 0; kw < kw_count; ++kw) {
+      const uint32_t w = bits[kw];
+      const float p = row[kw * 32 + lane];
+      s += ((w >> lane) & 1u) ? static_cast<double>(p) : -static_cast<double>(p);
+      row[kw * 32 + lane] = a * p;
+    }
+    s = warp_sum(s);
+    if (lane == 0) dalpha[j] = static_cast<float>(s);
+  }
+}
+
+// ---- P = dY^T X on the tensor cores ------------------------------------------------
+
+constexpr int kSsThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4..7 epilogue
+constexpr int kSsRowsA = 128;     // rows of X^T (k) per tile: the MMA's M
+constexpr int kSsRowsB = 256;     // rows of dY^T (j) per tile: the MMA's N
+constexpr int kSsUnit = 64;       // contraction (m) per stage: one 128-byte bf16 swizzle atom
+constexpr int kSsStages = 4;
+constexpr int kSsABytes = kSsRowsA * 128;
+constexpr int kSsBBytes = kSsRowsB * 128;
+constexpr int kSsStageBytes = kSsABytes + kSsBBytes;  // 48 KB
+constexpr int kSsSmemBytes = kSsStages * kSsStageBytes + 1024;
+
+// tm_a: X^T [Kdim][Mp] bf16, box 64 x 128; tm_b: dY^T [Ndim][Mp] bf16, box 64 x 256.
+// Writes P[j][k] (fp32, row pitch Kdim) for j < Ndim. Two accumulators in
+// tensor memory, so the epilogue of one tile overlaps the next tile's MMAs.
+__global__ void __launch_bounds__(kSsThreads, 1) gemm_ss_ste_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                                    const __grid_constant__ CUtensorMap tm_b,
+                                                                    int Kdim, int Ndim, int Mp,
+                                                                    float* __restrict__ P) {
+  extern __shared__ uint8_t ss_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ss_smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t full[kSsStages], empty[kSsStages], d_full[2], d_empty[2];
+  __shared__ uint32_t tmem_base_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_a = Kdim / kSsRowsA;
+  const int tiles_b = (Ndim + kSsRowsB - 1) / kSsRowsB;
+  const int num_tiles = tiles_a * tiles_b;
+  const int units = Mp / kSsUnit;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSsStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&d_full[b]), 1);
+      mbar_init(smem_u32(&d_empty[b]), 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_sh), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int k0 = (tile % tiles_a) * kSsRowsA, j0 = (tile / tiles_a) * kSsRowsB;
+        for (int u = 0; u < units; ++u, ++it) {
+          const uint32_t s = it % kSsStages;
+          if (it >= kSsStages && !mbar_wait(smem_u32(&empty[s]), ((it / kSsStages) - 1) & 1, kWhereSsProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_arrive_expect_tx(fb, kSsStageBytes);
+          uint8_t* st = smem + s * kSsStageBytes;
+          tma_load_2d(smem_u32(st), &tm_a, fb, u * kSsUnit, k0);
+          tma_load_2d(smem_u32(st + kSsABytes), &tm_b, fb, u * kSsUnit, j0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kSsRowsA, kSsRowsB);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tcount) {
+        const uint32_t ab = tcount & 1u;
+        if (tcount >= 2 && !mbar_wait(smem_u32(&d_empty[ab]), ((tcount / 2) - 1) & 1, kWhereSsMma)) break;
+        tc_fence_after_sync();
+        for (int u = 0; u < units; ++u, ++it) {
+          const uint32_t s = it % kSsStages;
+          if (!mbar_wait(smem_u32(&full[s]), (it / kSsStages) & 1, kWhereSsMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          uint8_t* st = smem + s * kSsStageBytes;
+          const uint64_t ad = sw128_kmajor_desc(smem_u32(st));
+          const uint64_t bd = sw128_kmajor_desc(smem_u32(st + kSsABytes));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // 16 bf16 = 32 bytes of the atom per MMA
+            umma_bf16(tmem + ab * kSsRowsB, ad + static_cast<uint64_t>(kk * 2), bd + static_cast<uint64_t>(kk * 2),
+                      idesc, (u > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&empty[s]));
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&d_full[ab]));
+      }
+    }
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+      const uint32_t ab = tcount & 1u;
+      const int k0 = (tile % tiles_a) * kSsRowsA, j0 = (tile / tiles_a) * kSsRowsB;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&d_full[ab]), (tcount / 2) & 1, kWhereSsEpilogue));
+      if (!ok) break;
+      tc_fence_after_sync();
+      const int k = k0 + q * 32 + lane;  // this thread's row of D = column of P
+#pragma unroll 1
+      for (int cc = 0; cc < kSsRowsB / 32; ++cc) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem + ab * kSsRowsB + cc * 32 + (static_cast<uint32_t>(q * 32) << 16), r);
+        tmem_wait_ld();
+        const int jc = j0 + cc * 32;
+        float* pp = P + static_cast<int64_t>(jc) * Kdim + k;
+        if (jc + 32 <= Ndim) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i, pp += Kdim) *pp = __uint_as_float(r[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i, pp += Kdim)
+            if (jc + i < Ndim) *pp = __uint_as_float(r[i]);
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&d_empty[ab]));
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bl

@@ -32,6 +32,9 @@ enum : int {
   kWhereLutInbox = 5,
   kWhereStackLevel = 6,  // a level waited for the previous one
   kWhereStackInbox = 7,
+  kWhereSsProducer = 8,  // the straight-through weight-gradient GEMM
+  kWhereSsMma = 9,
+  kWhereSsEpilogue = 10,
 };
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.

@@ -68,6 +68,7 @@ extern "C" {
 #define BL_OP_W158A8 5
 #define BL_OP_W1A8_EX 6 /* bitlinear_w1a8_ex with a per-tensor quantiser */
 #define BL_OP_W1A16_STACK 7 /* bin_linear_w1a16_stack (M, N, K ignored) */
+#define BL_OP_W1A16_BACKWARD 8 /* bin_linear_w1a16_backward */
 
 /* Library ABI version (this header: 1). */
 int bl_abi_version(void);
@@ -136,6 +137,27 @@ int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alp
 #define BL_FLAG_OVERLAP_PREVIOUS 1u
 int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
                         int64_t M, int64_t N, int64_t K, unsigned flags, void* stream);
+
+/*
+ * bin_linear_w1a16_backward -- gradients of the FBI-linear forward with the
+ * straight-through estimator ("FBI-LLM" page, FBI-linear paragraph: the
+ * estimator carries the gradient through the sign function; no clipping
+ * window is given, so ds/dW is taken as 1). With z = S x (before alpha) and
+ * the incoming gradient dy [M x N] bf16:
+ *   dx[m][k]  = bf16( sum_j dy[m][j] * alpha[j] * s_jk )
+ *   dw[j][k]  = alpha[j] * sum_m dy[m][j] * x[m][k]          (fp32)
+ *   dalpha[j] = sum_m dy[m][j] * z[m][j] = sum_k s_jk * sum_m dy[m][j] x[m][k]   (fp32)
+ * x [M x K] bf16, packed [N x K/32] and alpha [N] as in the forward. dx may
+ * be NULL (not computed); dw and dalpha are both given or both NULL. dx
+ * takes dy * alpha split into two bf16 parts through the forward kernels;
+ * the products over m run on the tensor cores with fp32 accumulation.
+ * K % 128 == 0 and N % 128 == 0. ws: bl_workspace_bytes(BL_OP_W1A16_BACKWARD,
+ * M, N, K) bytes of device memory, 16-byte aligned. M == 0 zero-fills dw and
+ * dalpha.
+ */
+int bin_linear_w1a16_backward(const uint16_t* x, const uint32_t* packed, const float* alpha,
+                              const uint16_t* dy, uint16_t* dx, float* dw, float* dalpha, int64_t M,
+                              int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * bin_linear_w1a16_stack -- single-token decode through a stack of FBI-linear

@@ -49,6 +49,7 @@ class Oracle:
             "oracle_w158a8_acc": [_p, _p, _i64, _i64, _i64, _p],
             "oracle_w158a8_acc_at": [_p, _p, _i64, _p, _p, _i64, _p],
             "oracle_w1a16_backward": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p],
+            "oracle_w1a16_backward_at": [_p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p, _p, _i64, _p],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -107,6 +108,26 @@ class Oracle:
         self._lib.oracle_w1a16_backward(_ptr(x), _ptr(packed), _ptr(alpha), _ptr(dy), M, N, K, _ptr(dx), _ptr(dw),
                                         _ptr(da))
         return dx, dw, da
+
+    def w1a16_backward_at(self, x_bf16, packed, alpha, dy_bf16, K: int, which: str, i0, i1=None):
+        """One of the backward outputs at positions: which = "dx" at (m, k) = (i0, i1),
+        "dw" at (j, k) = (i0, i1), "dalpha" at j = i0."""
+        x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+        dy = np.ascontiguousarray(dy_bf16, dtype=np.uint16)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        alpha = np.ascontiguousarray(alpha, dtype=np.float32)
+        M, N = dy.shape
+        assert x.shape == (M, K) and packed.shape == (N, self.row_words(K))
+        i0 = np.ascontiguousarray(i0, dtype=np.int64)
+        i1 = np.ascontiguousarray(np.zeros_like(i0) if i1 is None else i1, dtype=np.int64)
+        code = {"dx": 0, "dw": 1, "dalpha": 2}[which]
+        lim0 = M if code == 0 else N
+        assert i0.size == 0 or (i0.min() >= 0 and i0.max() < lim0)
+        assert code == 2 or i1.size == 0 or (i1.min() >= 0 and i1.max() < K)
+        out = np.zeros(i0.shape, dtype=np.float64)
+        self._lib.oracle_w1a16_backward_at(_ptr(x), _ptr(packed), _ptr(alpha), _ptr(dy), M, N, K, code, _ptr(i0),
+                                           _ptr(i1), i0.size, _ptr(out))
+        return out
 
     def w1a16_at(self, x_bf16, packed, alpha, K: int, ms, js):
         x = np.ascontiguousarray(x_bf16, dtype=np.uint16)

@@ -429,6 +429,37 @@ void oracle_w1a16_backward(const uint16_t* x, const uint32_t* packed, const floa
     }
 }
 
+/* the same definitions at a list of positions, for sampled checks of
+ * problems too large to compute whole: which = 0 gives dx at (m, k) =
+ * (i0, i1), 1 gives dw at (j, k) = (i0, i1), 2 gives dalpha at j = i0 */
+void oracle_w1a16_backward_at(const uint16_t* x, const uint32_t* packed, const float* alpha,
+                              const uint16_t* dy, int64_t M, int64_t N, int64_t K, int which,
+                              const int64_t* i0, const int64_t* i1, int64_t count, double* out)
+{
+    for (int64_t i = 0; i < count; ++i) {
+        double s = 0.0;
+        if (which == 0) {
+            const int64_t m = i0[i], k = i1[i];
+            for (int64_t j = 0; j < N; ++j)
+                s += bf16_value(dy[m * N + j]) * (double)alpha[j] * (double)packed_sign(packed, K, j, k);
+        } else if (which == 1) {
+            const int64_t j = i0[i], k = i1[i];
+            for (int64_t m = 0; m < M; ++m)
+                s += bf16_value(dy[m * N + j]) * bf16_value(x[m * K + k]);
+            s *= (double)alpha[j];
+        } else {
+            const int64_t j = i0[i];
+            for (int64_t m = 0; m < M; ++m) {
+                double z = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    z += (double)packed_sign(packed, K, j, k) * bf16_value(x[m * K + k]);
+                s += bf16_value(dy[m * N + j]) * z;
+            }
+        }
+        out[i] = s;
+    }
+}
+
 /* ---- W1A1 (only as an identity check of the packed-sign reading) ------- */
 
 /* dot_mj = sum_k a_mk * b_jk with both operands packed +-1 rows (R8);

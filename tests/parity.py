@@ -109,3 +109,28 @@ def guards_intact(buf: torch.Tensor, n: int, guard_elems=64, sentinel=None) -> b
     head = buf[:guard_elems]
     tail = buf[guard_elems + n:]
     return bool((head == sentinel).all().item() and (tail == sentinel).all().item())
+
+
+# ---- straight-through backward of the FBI-linear forward
+# dx (bf16): the W1A16 form with g = dy * alpha as the input:
+#   |dx - ref| <= 1e-4 * sum_j |dy_mj alpha_j|  +  half a bf16 ulp of (|ref| + that);
+# dw (fp32): |dw - ref| <= 1e-4 * |alpha_j| * sum_m |dy_mj x_mk|  +  one fp32 ulp of |ref|;
+# dalpha (fp32): |dalpha - ref| <= 1e-4 * sum_m |dy_mj| sum_k |x_mk|  +  one fp32 ulp of |ref|.
+def _f32_ulp(v: np.ndarray) -> np.ndarray:
+    a = np.abs(v)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.exp2(e - 23)
+
+
+def ste_dx_bound(dy_abs: np.ndarray, alpha: np.ndarray, ref: np.ndarray, ms) -> np.ndarray:
+    tol = W1A16_REL * (dy_abs @ np.abs(alpha.astype(np.float64)))[ms]
+    return tol + 0.5 * bf16_ulp(np.abs(ref) + tol)
+
+
+def ste_dw_bound(dy_abs: np.ndarray, x_abs: np.ndarray, alpha: np.ndarray, ref: np.ndarray, js, ks) -> np.ndarray:
+    s = np.einsum("mi,mi->i", dy_abs[:, js], x_abs[:, ks])
+    return W1A16_REL * np.abs(alpha.astype(np.float64))[js] * s + _f32_ulp(ref)
+
+
+def ste_dalpha_bound(dy_abs: np.ndarray, x_abs: np.ndarray, ref: np.ndarray, js) -> np.ndarray:
+    return W1A16_REL * (dy_abs[:, js].T @ x_abs.sum(axis=1)) + _f32_ulp(ref)

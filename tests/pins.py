@@ -543,6 +543,18 @@ def pin_backward_dw_ignores_signs(o):
     assert np.allclose(dw1, alpha.astype(np.float64)[:, None] * P, rtol=1e-13, atol=1e-13)
 
 
+def pin_backward_sampled_equals_full(o):
+    M, N, K = 3, 7, 96
+    W, x, dy = _backward_case(59, M, N, K)
+    packed, alpha = o.pack_fbi(W)
+    dx, dw, da = o.w1a16_backward(x, packed, alpha, dy, K)
+    ms, ks = np.meshgrid(np.arange(M), np.arange(K), indexing="ij")
+    assert np.array_equal(o.w1a16_backward_at(x, packed, alpha, dy, K, "dx", ms.ravel(), ks.ravel()), dx.ravel())
+    js, ks = np.meshgrid(np.arange(N), np.arange(K), indexing="ij")
+    assert np.array_equal(o.w1a16_backward_at(x, packed, alpha, dy, K, "dw", js.ravel(), ks.ravel()), dw.ravel())
+    assert np.array_equal(o.w1a16_backward_at(x, packed, alpha, dy, K, "dalpha", np.arange(N)), da)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]
 
 
