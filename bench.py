@@ -344,6 +344,101 @@ class Prefill(Workload):
             self.o.w1a16(x, p, a, K)
 
 
+class Backward(Workload):
+    """Straight-through backward of FBI-linear at the 7B MLP up-projection
+    shape (2048 tokens, 4096 -> 11008): dx, dW and dalpha per step."""
+    name = "backward"
+    M, K, N = 2048, 4096, 11008
+    metric = "FBI-linear STE backward TFLOP/s (dx + dW, 7B MLP up-projection, 2048 tokens)"
+    unit, scale, bound = "TFLOP/s", 1e12, "tensor"
+    kernel = ("gemm_ts_kernel<0,1,256,false> (dx on transposed signs) + gemm_ss_ste_kernel (dW) + "
+              "layout kernels (one call)")
+    sources = [CSRC + "bl_backward.cuh", CSRC + "bl_gemm_ts.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    launches_per_step = 8  # split, transposed pack, fill, dx GEMM, two transposes, dW GEMM, finalize
+    rotate = 2
+
+    def __init__(self):
+        M, K, N = self.M, self.K, self.N
+        per_copy = M * K * 2 + M * N * 2 + N * K // 8 + 4 * N + M * K * 2 + N * K * 4 + 4 * N
+        self.config = {"workload": "FBI-linear straight-through backward, 2048 tokens, 7B MLP up-projection "
+                                   "4096->11008 (dx bf16, dW fp32, dalpha fp32)",
+                       "M": M, "K": K, "N": N,
+                       "l2": f"inputs larger than L2: {self.rotate} distinct copies of x, dy, weights, gradients "
+                             f"and workspaces ({self.rotate * per_copy / 1e6:.0f} MB plus workspaces) rotated"}
+
+    def units_per_step(self):
+        return 2.0 * (2.0 * self.M * self.N * self.K)  # the dx and dW contractions
+
+    def peak(self, peaks, timed_s):
+        key = "bf16_tflops_sustained" if timed_s > SUSTAINED_AFTER_S else "bf16_tflops"
+        return peaks[key], key
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        from bit_linear_layers_b200 import synthetic
+        self.bl = bl
+        M, K, N = self.M, self.K, self.N
+        self.copies = []
+        for i in range(self.rotate):
+            seed = 3 + 100 * i + 7 * rank
+            W = synthetic.weights(N, K, seed=seed, device=dev)
+            p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
+            del W
+            x = synthetic.activations(M, K, seed=seed, device=dev)
+            dy = synthetic.activations(M, N, seed=seed + 1, device=dev)
+            dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+            dw = torch.empty((N, K), dtype=torch.float32, device=dev)
+            da = torch.empty(N, dtype=torch.float32, device=dev)
+            ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W1A16_BACKWARD, M, N, K), dtype=torch.uint8, device=dev)
+            self.copies.append((x, dy, p, a, dx, dw, da, ws))
+        c = self.copies[0]
+        self.xh, self.dyh = c[0].cpu().pin_memory(), c[1].cpu().pin_memory()
+        self.dxh = torch.empty_like(c[4], device="cpu").pin_memory()
+        self.dwh = torch.empty_like(c[5], device="cpu").pin_memory()
+        self.dah = torch.empty_like(c[6], device="cpu").pin_memory()
+        self.h2d = M * K * 2 + M * N * 2
+        self.d2h = M * K * 2 + N * K * 4 + N * 4
+
+    def step(self, i):
+        x, dy, p, a, dx, dw, da, ws = self.copies[i % self.rotate]
+        self.bl.bin_linear_w1a16_backward(x, p, a, dy, dx=dx, dw=dw, dalpha=da, ws=ws)
+
+    def e2e_step(self, i):
+        x, dy, p, a, dx, dw, da, ws = self.copies[i % self.rotate]
+        x.copy_(self.xh, non_blocking=True)
+        dy.copy_(self.dyh, non_blocking=True)
+        self.bl.bin_linear_w1a16_backward(x, p, a, dy, dx=dx, dw=dw, dalpha=da, ws=ws)
+        self.dxh.copy_(dx, non_blocking=True)
+        self.dwh.copy_(dw, non_blocking=True)
+        self.dah.copy_(da, non_blocking=True)
+
+    # oracle: 64 entries of dx and 64 of dW at the full shape per call
+    ORACLE_POINTS = 64
+
+    def oracle_setup(self):
+        import numpy as np
+        import oracle as oracle_pkg
+        from bit_linear_layers_b200 import synthetic
+        self.o = oracle_pkg.get()
+        M, K, N = self.M, self.K, self.N
+        W = synthetic.weights(N, K, seed=3).numpy()
+        self.op, self.oa = self.o.pack_fbi(W)
+        self.ox = synthetic.bf16_bits(synthetic.activations(M, K, seed=3))
+        self.ody = synthetic.bf16_bits(synthetic.activations(M, N, seed=4))
+        rng = np.random.default_rng(0)
+        n = self.ORACLE_POINTS
+        self.opts = (rng.integers(0, M, n), rng.integers(0, K, n), rng.integers(0, N, n), rng.integers(0, K, n))
+        self.oracle_sample = (f"{n} entries of dx (each a sum over the 11008 outputs) and {n} of dW (each a sum "
+                              "over the 2048 tokens) per call (single-threaded C oracle, fp64)")
+        return 2.0 * n * N + 2.0 * n * M
+
+    def oracle_call(self):
+        ms, ks, js, ks2 = self.opts
+        self.o.w1a16_backward_at(self.ox, self.op, self.oa, self.ody, self.K, "dx", ms, ks)
+        self.o.w1a16_backward_at(self.ox, self.op, self.oa, self.ody, self.K, "dw", js, ks2)
+
+
 class W1A8(Workload):
     name = "w1a8"
     SHAPES = [(512, 2048, 5632), (512, 5632, 2048)]
@@ -624,7 +719,7 @@ class W1A1(Workload):
             self.o.w1a1(a, b, K)
 
 
-WORKLOADS = {w.name: w for w in (Decode, Prefill, W1A8, W158A8, W1A8Tensor, W1A1)}
+WORKLOADS = {w.name: w for w in (Decode, Prefill, Backward, W1A8, W158A8, W1A8Tensor, W1A1)}
 
 
 # ----------------------------------------------------------------------------- ours
