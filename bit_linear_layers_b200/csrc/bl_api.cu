@@ -16,6 +16,7 @@
 #include "bl_gemm_ts.cuh"
 #include "bl_gemv.cuh"
 #include "bl_gemv_lut.cuh"
+#include "bl_gemv_mma.cuh"
 #include "bl_gemv_stack.cuh"
 #include "bl_lnquant.cuh"
 #include "bl_pack.cuh"
@@ -86,7 +87,11 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
               set_ts_smem<0>() && set_ts_smem<1>() && set_ts_smem<2>() &&
               set_smem(gemv_w1a16_stack_kernel, kStackPages * kLutPageBytes) &&
-              set_smem(gemm_ss_ste_kernel, kSsSmemBytes);
+              set_smem(gemm_ss_ste_kernel, kSsSmemBytes) &&
+              set_smem(gemv_w1a16_mma_kernel<8, 16>, mma_smem_bytes(8, 16)) &&
+              set_smem(gemv_w1a16_mma_kernel<16, 16>, mma_smem_bytes(16, 16)) &&
+              set_smem(gemv_w1a16_mma_kernel<8, kMmaMaxSliceWords>, mma_smem_bytes(8, kMmaMaxSliceWords)) &&
+              set_smem(gemv_w1a16_mma_kernel<16, kMmaMaxSliceWords>, mma_smem_bytes(16, kMmaMaxSliceWords));
     if (!ok) cudaGetLastError();
     {
       cudaLaunchConfig_t cfg = {};
@@ -194,6 +199,36 @@ int check_shape(int64_t M, int64_t N, int64_t K) {
   if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return BL_ERR_UNSUPPORTED;
   if (M * K >= kMaxProduct || N * K >= kMaxProduct || M * N >= kMaxProduct) return BL_ERR_UNSUPPORTED;
   return BL_OK;
+}
+
+// ---- few-token warp-MMA GEMV (5 <= M <= 16, K % 256 == 0, K <= 12288) ---------------
+template <int MT, int SWMAX>
+cudaError_t launch_mma_t(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y, int M,
+                         int N, int K, bool overlap, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kMmaCluster, static_cast<unsigned>(cdiv(N, kMmaRowsPerCluster)), 1);
+  cfg.blockDim = dim3(kMmaThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(mma_smem_bytes(MT, K / 256));
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = kMmaCluster;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = overlap ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, gemv_w1a16_mma_kernel<MT, SWMAX>, x, packed, alpha, y, M, N, K);
+}
+cudaError_t launch_mma(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y, int M, int N,
+                       int K, bool overlap, cudaStream_t s) {
+  const bool small_k = K / 256 <= 16;
+  if (M <= 8)
+    return small_k ? launch_mma_t<8, 16>(x, packed, alpha, y, M, N, K, overlap, s)
+                   : launch_mma_t<8, kMmaMaxSliceWords>(x, packed, alpha, y, M, N, K, overlap, s);
+  return small_k ? launch_mma_t<16, 16>(x, packed, alpha, y, M, N, K, overlap, s)
+                 : launch_mma_t<16, kMmaMaxSliceWords>(x, packed, alpha, y, M, N, K, overlap, s);
 }
 
 // ---- single-token lookup-table GEMV ------------------------------------------------
@@ -502,6 +537,15 @@ int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* 
       e = launch_lut<2>(x, packed, alpha, y, int(N), int(K), C, slice_words, overlap, s);
     else
       e = launch_lut<3>(x, packed, alpha, y, int(N), int(K), C, slice_words, overlap, s);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    return launch_status();
+  }
+  if (M > 4 && M <= 16 && K % 256 == 0 && K / 256 <= kMmaMaxSliceWords) {  // measured faster than tcgen05 here
+    const cudaError_t e = launch_mma(x, packed, alpha, y, int(M), int(N), int(K),
+                                     (flags & BL_FLAG_OVERLAP_PREVIOUS) != 0, s);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return BL_ERR_CUDA;

@@ -35,6 +35,7 @@ enum : int {
   kWhereSsProducer = 8,  // the straight-through weight-gradient GEMM
   kWhereSsMma = 9,
   kWhereSsEpilogue = 10,
+  kWhereMmaInbox = 11,  // the few-token warp-MMA GEMV
 };
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.

@@ -42,8 +42,12 @@ FULL = [
     (1, 4099, 384), (1, 77, 8320),
     # few-token GEMV path (M <= 4)
     (2, 300, 384), (3, 129, 256), (4, 1000, 11008),
+    # 5..16 tokens, K % 256 == 0: warp-MMA GEMV (8- and 16-token tiles, 16- and 48-word slices,
+    # slices shorter than a word group, ragged row clusters)
+    (6, 384, 256), (8, 1000, 4096), (9, 129, 2048), (12, 4099, 512), (16, 300, 4096), (16, 257, 11008),
+    (7, 200, 12288), (13, 128, 8192),
     # tcgen05 GEMM path
-    (5, 384, 256), (16, 128, 128), (17, 200, 384), (129, 383, 640), (256, 512, 1024),
+    (5, 384, 384), (16, 128, 128), (17, 200, 384), (129, 383, 640), (256, 512, 1024),
     (300, 1000, 1024), (1000, 1100, 512),
     # enough tiles for the 128-row x 256-token configuration, ragged in M and N
     (300, 9100, 256),
