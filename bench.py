@@ -445,7 +445,7 @@ class W1A8(Workload):
     metric = "BitLinear W1A8 TOP/s (1.3B shapes, 512 tokens, LN + absmax quant + int8 GEMM + rescale)"
     unit, scale, bound = "TOP/s", 1e12, "tensor"
     dtype = "s8"
-    kernel = "ln_quant_kernel + gemm_ts_kernel<1,2,128,*> (one call; time includes LN + quantisation)"
+    kernel = "ln_quant_kernel<NV> + gemm_ts_kernel<1,1,256|128,*> (one call; time includes LN + quantisation)"
     sources = [CSRC + "bl_gemm_ts.cuh", CSRC + "bl_lnquant.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
     traffic_file = "bitlinear_w1a8_1p3b_512tokens.traffic.json"  # the GEMM launches' DRAM bytes
     launches_per_step = 4
@@ -532,7 +532,7 @@ class W158A8(W1A8):
     W / mean|W|, two bit planes)."""
     name = "w158a8"
     metric = "BitLinear b1.58 W1.58A8 TOP/s (1.3B shapes, 512 tokens, ternary weights)"
-    kernel = "ln_quant_kernel + gemm_ts_kernel<2,1,T,*> (one call; time includes LN + quantisation)"
+    kernel = "ln_quant_kernel<NV> + gemm_ts_kernel<2,1,T,*> (one call; time includes LN + quantisation)"
     traffic_file = None
 
     def __init__(self):

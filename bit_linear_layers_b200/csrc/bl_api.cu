@@ -383,7 +383,15 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
     int8_t* xq_ws = static_cast<int8_t*>(ws);
     double* g_ws = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(size_t(M * K)));
     if (!quant) {
-      ln_quant_kernel<<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
+      const int64_t nv = cdiv(K / 8, kLnThreads);  // 16-byte vectors per thread
+      if (nv <= 1)
+        ln_quant_kernel<1><<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
+      else if (nv <= 2)
+        ln_quant_kernel<2><<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
+      else if (nv <= 4)
+        ln_quant_kernel<4><<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
+      else
+        ln_quant_kernel<0><<<static_cast<unsigned>(M), kLnThreads, 0, s>>>(x, M, K, xq_ws, g_ws);
       if ((rc = launch_status()) != BL_OK) return rc;
     } else {
       const bool nonneg = (quant & BL_W1A8_NONNEG) != 0;

@@ -87,6 +87,10 @@ __device__ __forceinline__ double ln_block_sum(double v, double* sh) {
   return t;
 }
 
+// NV > 0: the token's row is loaded once into registers (at most NV 16-byte
+// vectors per thread, K <= NV * 2048) and the three passes read it from
+// there; NV = 0: every pass streams the row again (any K).
+template <int NV>
 __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                               int64_t K, int8_t* __restrict__ xq,
                                                               double* __restrict__ gamma_out) {
@@ -97,11 +101,31 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
   const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
   const int64_t nvec = K / 8;  // 8 bf16 per 16-byte load
 
+  uint4 cache[NV > 0 ? NV : 1];
+  if constexpr (NV > 0) {
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+      const int64_t i = threadIdx.x + static_cast<int64_t>(u) * kLnThreads;
+      cache[u] = i < nvec ? row[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  // f(i, v) for every 16-byte vector i of the row this thread owns
+  auto for_each_vec = [&](auto&& f) {
+    if constexpr (NV > 0) {
+#pragma unroll
+      for (int u = 0; u < NV; ++u) {
+        const int64_t i = threadIdx.x + static_cast<int64_t>(u) * kLnThreads;
+        if (i < nvec) f(i, cache[u]);
+      }
+    } else {
+      for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) f(i, row[i]);
+    }
+  };
+
   // pass 1: fp64 sum (two chains), fp32 max and min
   double s0 = 0.0, s1 = 0.0;
   float xmax = -INFINITY, xmin = INFINITY;
-  for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
-    const uint4 v = row[i];
+  for_each_vec([&](int64_t, const uint4& v) {
     const uint32_t h[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -111,7 +135,7 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
       xmax = fmaxf(xmax, fmaxf(a, b));
       xmin = fminf(xmin, fminf(a, b));
     }
-  }
+  });
   xmax = warp_max(xmax);
   xmin = -warp_max(-xmin);
   if ((threadIdx.x & 31) == 0) {
@@ -129,8 +153,7 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
 
   // pass 2: sum of squared deviations in fp64
   double q0 = 0.0, q1 = 0.0;
-  for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
-    const uint4 v = row[i];
+  for_each_vec([&](int64_t, const uint4& v) {
     const uint32_t h[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -139,7 +162,7 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
       q0 = fma(d0, d0, q0);
       q1 = fma(d1, d1, q1);
     }
-  }
+  });
   const double sq = ln_block_sum(q0 + q1, sh);
   const double dmax = fmax(static_cast<double>(xmax) - mu, mu - static_cast<double>(xmin));
   LnQuantParams p;
@@ -151,10 +174,9 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
   p.c32 = dmax > 0.0 ? static_cast<float>(128.0 / dmax) : 0.f;
   if (threadIdx.x == 0) gamma_out[m] = p.gamma;
 
-  // pass 3: codes, 8 per thread per step
+  // pass 3: codes, 8 per thread per vector
   uint2* out = reinterpret_cast<uint2*>(xq + m * K);
-  for (int64_t i = threadIdx.x; i < nvec; i += kLnThreads) {
-    const uint4 v = row[i];
+  for_each_vec([&](int64_t i, const uint4& v) {
     const uint32_t h[4] = {v.x, v.y, v.z, v.w};
     uint32_t packed_codes[2] = {0u, 0u};
     if (dmax > 0.0) {
@@ -167,7 +189,7 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
       }
     }
     out[i] = make_uint2(packed_codes[0], packed_codes[1]);
-  }
+  });
 }
 
 // ---------------------------------------------------------------------------
