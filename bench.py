@@ -354,6 +354,7 @@ class Backward(Workload):
     kernel = ("gemm_ts_kernel<0,1,256,false> (dx on transposed signs) + gemm_ss_ste_kernel (dW) + "
               "layout kernels (one call)")
     sources = [CSRC + "bl_backward.cuh", CSRC + "bl_gemm_ts.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = "ste_backward_2048x4096x11008.traffic.json"  # the dx GEMM launch (largest share of the step)
     launches_per_step = 8  # split, transposed pack, fill, dx GEMM, two transposes, dW GEMM, finalize
     rotate = 2
 
