@@ -12,11 +12,10 @@
 //     kernel (byte tables of the slice in shared memory, one PRMT + LDS + FADD
 //     per 8 weights) and sweep 256-row blocks, block b of a level going to
 //     cluster b % G;
-//   * the packed words of a CTA's next block are loaded into registers while
-//     it computes the current one, and those of its first block of a level are
-//     loaded before it waits for the level's input; the rows of its next
-//     level are prefetched into L2 at the start of each level, so the weight
-//     stream does not stop at the level boundaries;
+//   * the packed words of a pass (up to 4 blocks) are loaded into registers
+//     before the lookups, and those of a level's first pass before the CTA
+//     waits for the level's input (prefetching the next level into L2, with
+//     per-line or bulk prefetches, measured no faster and is not done);
 //   * levels are separated by a grid-wide completion count: every CTA adds 1
 //     (release, GPU scope) once its outputs of level l are written, and a CTA
 //     reads the input of level l + 1 only after the count of level l reached
@@ -78,31 +77,11 @@ __device__ __forceinline__ void cluster_arrive_release() {
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // the linear of level `lv` that block b falls in
 __device__ __forceinline__ const StackJob& stack_job_of(const StackParams& P, const StackLevel& lv, int b) {
   int j = lv.job0;
   while (j + 1 < lv.job0 + lv.njobs && b >= P.jb[j + 1].block0) ++j;
   return P.jb[j];
-}
-
-// Bring this CTA's slice of the rows of its blocks of level l into L2 (one
-// prefetch per touched 128-byte line, spread over the CTA's threads).
-__device__ __forceinline__ void stack_prefetch_level(const StackParams& P, int l, uint32_t rank) {
-  const StackLevel& lv = P.lv[l];
-  const int words = lv.K / 32, slice_words = words / kStackCluster;
-  for (int b = blockIdx.y; b < lv.nblocks; b += gridDim.y) {
-    const StackJob& jb = stack_job_of(P, lv, b);
-    const int row = (b - jb.block0) * kLutRowsPerCluster + static_cast<int>(threadIdx.x);
-    if (row >= jb.N) continue;
-    const uint32_t* w = jb.packed + static_cast<int64_t>(row) * words + static_cast<int>(rank) * slice_words;
-    const uintptr_t first = reinterpret_cast<uintptr_t>(w) & ~static_cast<uintptr_t>(127);
-    const uintptr_t last = (reinterpret_cast<uintptr_t>(w + slice_words) - 1) & ~static_cast<uintptr_t>(127);
-    for (uintptr_t a = first; a <= last; a += 128) prefetch_l2(reinterpret_cast<const void*>(a));
-  }
 }
 
 // Blocks of one level held in registers at once, per table page count.
@@ -149,7 +128,6 @@ __device__ __forceinline__ void stack_level(const StackParams& P, int l, uint32_
 
   // the first pass's words do not depend on x: load them before waiting
   if (my_blocks > 0) load_pass(0);
-  if (l + 1 < P.num_levels) stack_prefetch_level(P, l + 1, rank);
 
   // the input of this level is complete once every CTA has finished level l - 1
   if (l > 0) {
@@ -242,7 +220,6 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_w1a16_stack_kernel(const 
 
   uint32_t n = 0;
   bool waiting = true;
-  if (P.num_levels > 0) stack_prefetch_level(P, 0, rank);
   for (int l = 0; l < P.num_levels; ++l) {
     const int slice_words = P.lv[l].K / (32 * kStackCluster);
     if (slice_words <= 16)
