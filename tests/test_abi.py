@@ -104,6 +104,22 @@ def test_stack_validation_without_device_work():
     assert call(4096, x=ODD.value) == -1
 
 
+def test_backward_validation_without_device_work():
+    import bit_linear_layers_b200 as bl
+    ws = bl.workspace_bytes(bl.BL_OP_W1A16_BACKWARD, 64, 256, 256)
+    # g = [hi | lo] (64 x 512 bf16), S^T twice, K scales, x^T and dy^T with M padded to 64
+    assert ws >= 64 * 256 * 4 + 256 * 256 // 4 + 256 * 4 + 256 * 64 * 2 + 256 * 64 * 2
+
+    def call(M, N, K, dw=FAKE, dalpha=FAKE, ws_bytes=1 << 30, x=FAKE):
+        return bl.lib.bin_linear_w1a16_backward(x, FAKE, FAKE, FAKE, FAKE, dw, dalpha, M, N, K, FAKE, ws_bytes, None)
+
+    assert call(4, 192, 256) == -2          # N % 128 != 0
+    assert call(4, 256, 200) == -2          # K % 128 != 0
+    assert call(4, 256, 256, dalpha=None) == -1  # dW and dalpha come together
+    assert call(4, 256, 256, ws_bytes=16) == -1
+    assert call(4, 256, 256, x=ODD) == -1
+
+
 def test_zero_tokens_is_a_noop():
     import bit_linear_layers_b200 as bl
     assert bl.lib.bin_linear_w1a16(None, FAKE, FAKE, None, 0, 128, 128, None) == 0
