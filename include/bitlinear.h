@@ -118,8 +118,9 @@ int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, f
  * only initialises them), y [M x N] bf16 (round to nearest even).
  * Accumulation is fp32. A single token uses a lookup-table GEMV (a cluster
  * of CTAs splits K; signed byte sums of x are tabulated in shared memory);
- * up to 4 tokens a predicated-add GEMV; more tokens a tcgen05 tensor-core
- * GEMM. No workspace.
+ * up to 4 tokens a predicated-add GEMV; 5 to 16 tokens (K % 256 == 0,
+ * K <= 12288) a GEMV whose products run on the warp-level MMA; more tokens a
+ * tcgen05 tensor-core GEMM. No workspace.
  */
 int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
                      int64_t M, int64_t N, int64_t K, void* stream);
