@@ -534,7 +534,7 @@ class W158A8(W1A8):
     name = "w158a8"
     metric = "BitLinear b1.58 W1.58A8 TOP/s (1.3B shapes, 512 tokens, ternary weights)"
     kernel = "ln_quant_kernel<NV> + gemm_ts_kernel<2,1,T,*> (one call; time includes LN + quantisation)"
-    traffic_file = None
+    traffic_file = "bitlinear_w158a8_1p3b_512tokens.traffic.json"
 
     def __init__(self):
         super().__init__()
@@ -597,7 +597,7 @@ class W1A8Tensor(W1A8):
     metric = "BitLinear W1A8 TOP/s, per-tensor activation gamma (1.3B shapes, 512 tokens)"
     kernel = ("ln_stats_kernel + ln_tensor_scalars_kernel + ln_quant_tensor_kernel + gemm_ts_kernel<1,*> "
               "(one call; time includes LN + quantisation)")
-    traffic_file = None
+    traffic_file = "bitlinear_w1a8_tensor_1p3b_512tokens.traffic.json"
     launches_per_step = 8
 
     def __init__(self):
@@ -648,6 +648,7 @@ class W1A1(Workload):
     dtype = "b1"
     kernel = "xnor_gemm_kernel (64x64 tiles, XOR + POPC on the integer pipes)"
     sources = [CSRC + "bl_xnor.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = "xnor_w1a1_1p3b_512tokens.traffic.json"
     launches_per_step = 2
     rotate = 8
     # 16 population counts per SM per clock (each one 32 +-1 products), 2 ops
