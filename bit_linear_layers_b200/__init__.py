@@ -10,6 +10,10 @@ if the library is missing, importing the binding raises.
     bin_linear_w1a16(x, packed, alpha)     -> y (bf16)
     bitlinear_w1a8(x, packed, beta)        -> y (fp32)
     bitlinear_w158a8(x, packed, beta)      -> y (fp32), b1.58 ternary weights
+    bitlinear_w1a8_ex(x, packed, beta, f)  -> y (fp32), per-tensor / Eq.(6) quantisers
+    bin_xnor_gemm(a, b, K)                 -> dot (int32), W1A1
+    bin_linear_w1a16_backward(x, packed, alpha, dy) -> dx, dW, dalpha (straight-through)
+    W1A16Stack(levels).run()               decode through a stack of layers in one launch
 """
 from __future__ import annotations
 
@@ -50,11 +54,7 @@ BL_W1A8_TERNARY = 1
 BL_W1A8_PER_TENSOR = 2
 BL_W1A8_NONNEG = 4
 
-# every symbol include/bitlinear.h declares, with its ctypes signature
-_i64 = ctypes.c_int64
-_p = ctypes.c_void_p
-_int = ctypes.c_int
-_sz = ctypes.c_size_t
+
 class StackJob(ctypes.Structure):
     """bl_stack_job: one linear of a stack level."""
     _fields_ = [("packed", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("y", ctypes.c_void_p),
@@ -67,6 +67,11 @@ class StackLevel(ctypes.Structure):
                 ("num_jobs", ctypes.c_int32)]
 
 
+# every symbol include/bitlinear.h declares, with its ctypes signature
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+_int = ctypes.c_int
+_sz = ctypes.c_size_t
 SIGNATURES = {
     "bl_abi_version": ([], _int),
     "bl_status_string": ([_int], ctypes.c_char_p),
