@@ -543,6 +543,25 @@ def pin_backward_dw_ignores_signs(o):
     assert np.allclose(dw1, alpha.astype(np.float64)[:, None] * P, rtol=1e-13, atol=1e-13)
 
 
+def pin_backward_example_e(o):
+    # hand-worked 2 x 3 x 4 example (tests/golden/ste_example_e.json), every value exact
+    ex = _load("ste_example_e.json")
+    W = np.array([[float(_frac(v)) for v in row] for row in ex["W"]], dtype=np.float32)
+    packed, _ = o.pack_fbi(W)
+    assert packed[:, 0].tolist() == ex["packed"], packed[:, 0].tolist()
+    alpha = np.array([float(_frac(a)) for a in ex["alpha"]], dtype=np.float32)
+    x = np.stack([_bf16_bits_of([_frac(v) for v in row]) for row in ex["x"]])
+    dy = np.stack([_bf16_bits_of([_frac(v) for v in row]) for row in ex["dy"]])
+    dx, dw, da = o.w1a16_backward(x, packed, alpha, dy, 4)
+    assert [[Fraction(float(v)) for v in r] for r in dx] == [[_frac(v) for v in r] for r in ex["dx"]], dx
+    assert [[Fraction(float(v)) for v in r] for r in dw] == [[_frac(v) for v in r] for r in ex["dW"]], dw
+    assert [Fraction(float(v)) for v in da] == [_frac(v) for v in ex["dalpha"]], da
+    # and the forward of the same layer gives alpha * z
+    y = o.w1a16(x, packed, alpha, 4)
+    want = [[_frac(a) * _frac(z) for a, z in zip(ex["alpha"], row)] for row in ex["z"]]
+    assert [[Fraction(float(v)) for v in r] for r in y] == want, y
+
+
 def pin_backward_sampled_equals_full(o):
     M, N, K = 3, 7, 96
     W, x, dy = _backward_case(59, M, N, K)
