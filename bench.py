@@ -209,7 +209,7 @@ class Decode(Workload):
     def setup(self, dev, rank):
         import torch
         import bit_linear_layers_b200 as bl
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.bl = bl
         self.packs, self.alphas, self.xs = [], [], []
         for i in range(self.rotate):
@@ -249,7 +249,7 @@ class Decode(Workload):
 
     def oracle_setup(self):
         import oracle as oracle_pkg
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.o = oracle_pkg.get()
         W = synthetic.weights(self.N, self.K, seed=2).numpy()
         self.ox = synthetic.bf16_bits(synthetic.activations(self.M, self.K, seed=2))
@@ -292,7 +292,7 @@ class Prefill(Workload):
     def setup(self, dev, rank):
         import torch
         import bit_linear_layers_b200 as bl
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.bl = bl
         self.copies = []
         for i in range(self.rotate):
@@ -326,7 +326,7 @@ class Prefill(Workload):
 
     def oracle_setup(self):
         import oracle as oracle_pkg
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.o = oracle_pkg.get()
         self.olayers, flop = [], 0.0
         for s, ((M, K, N), cols) in enumerate(zip(self.SHAPES, self.ORACLE_COLS)):
@@ -377,7 +377,7 @@ class Backward(Workload):
     def setup(self, dev, rank):
         import torch
         import bit_linear_layers_b200 as bl
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.bl = bl
         M, K, N = self.M, self.K, self.N
         self.copies = []
@@ -420,7 +420,7 @@ class Backward(Workload):
     def oracle_setup(self):
         import numpy as np
         import oracle as oracle_pkg
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.o = oracle_pkg.get()
         M, K, N = self.M, self.K, self.N
         W = synthetic.weights(N, K, seed=3).numpy()
@@ -469,7 +469,7 @@ class W1A8(Workload):
     def setup(self, dev, rank):
         import torch
         import bit_linear_layers_b200 as bl
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.bl = bl
         self.copies = []
         for i in range(self.rotate):
@@ -510,7 +510,7 @@ class W1A8(Workload):
 
     def oracle_setup(self):
         import oracle as oracle_pkg
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.o = oracle_pkg.get()
         self.olayers, ops = [], 0.0
         for s, (M, K, N) in enumerate(self.SHAPES):
@@ -545,7 +545,7 @@ class W158A8(W1A8):
     def setup(self, dev, rank):
         import torch
         import bit_linear_layers_b200 as bl
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.bl = bl
         self.copies = []
         for i in range(self.rotate):
@@ -570,7 +570,7 @@ class W158A8(W1A8):
 
     def oracle_setup(self):
         import oracle as oracle_pkg
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.o = oracle_pkg.get()
         self.olayers, ops = [], 0.0
         for s, (M, K, N) in enumerate(self.SHAPES):
@@ -614,7 +614,7 @@ class W1A8Tensor(W1A8):
 
     def oracle_setup(self):
         import oracle as oracle_pkg
-        from bit_linear_layers_b200 import synthetic
+        import synthetic
         self.o = oracle_pkg.get()
         self.olayers, ops = [], 0.0
         for s, (M, K, N) in enumerate(self.SHAPES):
@@ -855,7 +855,7 @@ def secondary_llama7b(dev, peaks):
     of one step, and a 4096-token prefill."""
     import torch
     import bit_linear_layers_b200 as bl
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     layers = []
     for layer in range(synthetic.LLAMA7B_LAYERS):
         mats = []
@@ -996,7 +996,7 @@ def secondary_pack(dev, peaks):
     modes: GB/s on the bytes it must move (W read, packed bits and scales written)."""
     import torch
     import bit_linear_layers_b200 as bl
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     N, K = 11008, 4096
     W = synthetic.weights(N, K, seed=6, device=dev)
     res = {}
@@ -1025,7 +1025,7 @@ def secondary_decode_warm(dev):
     programmatic dependent launch."""
     import torch
     import bit_linear_layers_b200 as bl
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(4096, 4096, seed=2, device=dev)
     p, a = bl.bin_pack(W, bl.BL_PACK_FBI)
     x = synthetic.activations(1, 4096, seed=2, device=dev)

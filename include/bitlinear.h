@@ -257,7 +257,9 @@ int bitlinear_w158a8_debug(const uint16_t* x, const uint32_t* packed, const floa
  *                       max(LN - eta), codes clamp(rne((LN - eta) * 128 /
  *                       gamma), 0, 127); the output is Eq.(7) as printed,
  *                       y = acc * beta * gamma / 128 (no eta term appears on
- *                       the page). Implies per tensor.
+ *                       the page). So y estimates beta * W~ (LN - eta), not
+ *                       beta * W~ LN: the eta * beta * sum_k W~_jk term is
+ *                       not added back. Implies per tensor.
  *   BL_W1A8_TERNARY     packed holds b1.58 ternary weights (BL_PACK_TERNARY).
  * With neither quantiser flag this is bitlinear_w1a8 (or w158a8). Codes are
  * decided in fp64 in the order of the formula. ws: bl_workspace_bytes(

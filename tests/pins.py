@@ -316,6 +316,13 @@ def pin_sampled_equals_full(o):
     xq, _ = o.ln_absmax_quant(x)
     acc = o.w1a8_acc(xq, packed, 64)
     assert np.array_equal(o.w1a8_acc_at(xq, packed, 64, ms, js), acc[ms, js])
+    # the ternary sampler against its full product (M != N, and no sample
+    # lies on the diagonal, so swapped token and output indices show)
+    Wt, xt = _random_case(62, 9, 128, M=5)
+    packed_t, _ = o.pack_ternary(Wt)
+    xq_t, _ = o.ln_absmax_quant(xt)
+    acc_t = o.w158a8_acc(xq_t, packed_t, 128)
+    assert np.array_equal(o.w158a8_acc_at(xq_t, packed_t, 128, ms, js), acc_t[ms, js])
 
 
 # ---- b1.58 ternary weights (BitNet b1.58 page, section 2, Eq.(9)-(11)) ----

@@ -20,7 +20,7 @@ def bl():
 
 
 def _case(oracle, M, N, K, seed):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, seed)
     x = synthetic.activations(M, K, seed)
     dy = synthetic.activations(M, N, seed + 7)
@@ -44,7 +44,7 @@ FULL = [(1, 128, 128), (3, 256, 384), (17, 384, 256), (64, 128, 640), (100, 640,
 
 @pytest.mark.parametrize("M,N,K", FULL)
 def test_backward_full(bl, oracle, M, N, K):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     x, dy, packed, alpha = _case(oracle, M, N, K, seed=M + N + K)
     xb, dyb = synthetic.bf16_bits(x), synthetic.bf16_bits(dy)
     dx_ref, dw_ref, da_ref = oracle.w1a16_backward(xb, packed, alpha, dyb, K)
@@ -63,7 +63,7 @@ def test_backward_full(bl, oracle, M, N, K):
 
 
 def test_backward_7b_mlp_sampled(bl, oracle):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     M, N, K = 2048, 11008, 4096
     x, dy, packed, alpha = _case(oracle, M, N, K, seed=1)
     xb, dyb = synthetic.bf16_bits(x), synthetic.bf16_bits(dy)
@@ -85,7 +85,7 @@ def test_backward_7b_mlp_sampled(bl, oracle):
 
 
 def test_backward_parts_and_empty_batch(bl, oracle):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     M, N, K = 40, 256, 256
     x, dy, packed, alpha = _case(oracle, M, N, K, seed=9)
     dp, da_dev = torch.from_numpy(packed.view(np.int32)).cuda(), torch.from_numpy(alpha).cuda()

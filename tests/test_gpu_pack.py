@@ -17,7 +17,7 @@ def bl():
 
 
 def _weights(N, K, seed, mean=0.0):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     return synthetic.weights(N, K, seed, mean=mean)
 
 

@@ -22,7 +22,7 @@ def bl():
 
 @pytest.mark.parametrize("N,K", [(1, 128), (3, 256), (257, 384), (1000, 1024), (4096, 4096)])
 def test_pack_ternary(bl, oracle, N, K):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, seed=N + K, mean=0.001)
     packed_ref, gamma_ref = oracle.pack_ternary(W.numpy())
     packed, buf, sent = guarded_empty((N, K // 16), torch.int32, "cuda")
@@ -39,7 +39,7 @@ def test_pack_ternary(bl, oracle, N, K):
 
 
 def _run(bl, oracle, M, N, K, seed, full=True):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, seed, mean=0.001)
     x = synthetic.laplace_channel_activations(M, K, seed)
     packed, gamma_w = oracle.pack_ternary(W.numpy())
@@ -88,7 +88,7 @@ def test_w158a8_1p3b_sampled(bl, oracle, M, N, K):
 
 def test_w158a8_unit_codes_give_plane_counts(bl):
     # codes all 1 (xq_in): acc_j = #(+1) - #(-1) of row j, from the planes
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     M, N, K = 40, 700, 640
     W = synthetic.weights(N, K, 9, mean=0.001, device="cuda")
     packed, beta = bl.bin_pack(W, bl.BL_PACK_TERNARY)
@@ -106,7 +106,7 @@ def test_w158a8_unit_codes_give_plane_counts(bl):
 
 def test_w158a8_end_to_end_pack_then_forward(bl, oracle):
     # bin_pack on the GPU feeding the forward, against the oracle's pack + forward
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     M, N, K = 64, 512, 1024
     W = synthetic.weights(N, K, 21, mean=0.001)
     x = synthetic.laplace_channel_activations(M, K, 21)

@@ -40,7 +40,7 @@ def test_xnor_gemm(bl, oracle, M, N, K):
 def test_xnor_gemm_extremes_and_packed_activations(bl, oracle):
     # identical rows give +K, complementary rows -K; and activations packed by
     # bin_pack (sign of x, Sign(0) = -1) through the same path
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     K = 512
     rng = np.random.default_rng(3)
     a = _rows(rng, 4, K)

@@ -19,14 +19,14 @@ def bl():
 
 
 def _case(M, N, K, seed):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, seed)
     x = synthetic.activations(M, K, seed)
     return W, x
 
 
 def _oracle_inputs(oracle, W, x):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     packed, alpha = oracle.pack_fbi(W.numpy())
     return packed, alpha, synthetic.bf16_bits(x)
 
@@ -106,7 +106,7 @@ def test_w1a16_learned_alpha_any_sign(bl, oracle):
 def test_w1a16_all_ones_closed_form(bl):
     # y_j = alpha_j * (#pos - #neg), independent of the oracle
     N, K = 384, 1024
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, 11).cuda()
     packed, alpha = bl.bin_pack(W, bl.BL_PACK_FBI)
     pos = (W > 0).sum(dim=1).float()
@@ -132,7 +132,7 @@ def test_w1a16_end_to_end_pack_then_linear(bl, oracle):
 
 def test_w1a16_negation_and_zero_tokens(bl):
     M, N, K = 33, 256, 256
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, 2).cuda()
     x = synthetic.activations(M, K, 2).cuda()
     packed, alpha = bl.bin_pack(W, bl.BL_PACK_FBI)
@@ -147,7 +147,7 @@ def test_w1a16_negation_and_zero_tokens(bl):
 def test_w1a16_overlap_flag_chain(bl, oracle):
     """BL_FLAG_OVERLAP_PREVIOUS on a chain of dependent single-token calls
     (each output is the next input): results must equal the oracle's."""
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     N = K = 2048
     layers = 6
     Ws = [synthetic.weights(N, K, 100 + i) for i in range(layers)]
@@ -160,7 +160,7 @@ def test_w1a16_overlap_flag_chain(bl, oracle):
         h = bl.bin_linear_w1a16(h, dp, da, flags=bl.BL_FLAG_OVERLAP_PREVIOUS)
         outs.append(h)
     torch.cuda.synchronize()
-    from bit_linear_layers_b200.synthetic import bf16_bits
+    from synthetic import bf16_bits
     xin = bf16_bits(x)
     for i, ((p, a), y) in enumerate(zip(refs, outs)):
         y_ref = oracle.w1a16(xin, p, a, K)
@@ -177,7 +177,7 @@ def test_w1a16_overlap_flag_chain_gemm(bl, M):
     calls that ping-pongs between two buffers, so every layer also overwrites
     the buffer the layer before it read. The results must equal, bit for bit,
     the same chain run without the flag."""
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     N = K = 1024
     layers = 6
     dev = []

@@ -28,7 +28,7 @@ def bl():
 
 
 def _linear(oracle, N, K, seed):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, seed)
     packed, alpha = oracle.pack_fbi(W.numpy())
     return (torch.from_numpy(packed.view(np.int32)).cuda(), torch.from_numpy(alpha).cuda(), packed, alpha)
@@ -36,7 +36,7 @@ def _linear(oracle, N, K, seed):
 
 def _check_level(oracle, x_dev, linears, what):
     """linears: (packed_np, alpha_np, y_dev) of one level; x_dev the level input."""
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     xb = synthetic.bf16_bits(x_dev.reshape(1, -1))
     K = xb.shape[1]
     for i, (packed, alpha, y) in enumerate(linears):
@@ -49,7 +49,7 @@ def _check_level(oracle, x_dev, linears, what):
 def _run_and_check(bl, oracle, spec, seed0):
     """spec: list of levels, each (K, [N...], src) where src is None (a fresh
     input) or (level, linear) whose output feeds this level."""
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     levels, host, outs = [], [], []
     for li, (K, Ns, src) in enumerate(spec):
         if src is None:
@@ -98,7 +98,7 @@ def test_stack_chained_levels(bl, oracle):
 
 def test_stack_matches_layer_by_layer_at_7b_shapes(bl, oracle):
     """K = 4096 and 11008 split 8 ways in both calls: identical bits."""
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     shapes = [(4096, 4096), (4096, 4096), (4096, 11008), (11008, 4096)]  # (K, N)
     x0 = synthetic.activations(1, 4096, 5).reshape(4096).cuda()
     mats = [_linear(oracle, N, K, 20 + i)[:2] for i, (K, N) in enumerate(shapes)]
@@ -118,7 +118,7 @@ def test_stack_matches_layer_by_layer_at_7b_shapes(bl, oracle):
 
 def test_stack_longer_than_one_launch(bl, oracle):
     # 140 levels (two launches), alternating between two buffers
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     K = N = 512
     dp, da, packed, alpha = _linear(oracle, N, K, 77)
     x0 = synthetic.activations(1, K, 78).reshape(K).cuda()
@@ -134,7 +134,7 @@ def test_stack_longer_than_one_launch(bl, oracle):
 
 def test_stack_many_linears_per_launch(bl, oracle):
     # 300 linears over 3 levels (more than 256 linears: split between launches)
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     K = 256
     dp, da, packed, alpha = _linear(oracle, 64, K, 90)
     xs = [synthetic.activations(1, K, 91 + i).reshape(K).cuda() for i in range(3)]

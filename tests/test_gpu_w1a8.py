@@ -22,7 +22,7 @@ def bl():
 
 
 def _case(M, N, K, seed, kind="laplace_channel", w_mean=0.001):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, seed, mean=w_mean)
     x = synthetic.make_x(kind, M, K, seed)
     return W, x
@@ -42,7 +42,7 @@ def _check_codes(oracle, xb, xq_gpu, gamma_gpu):
 
 
 def _run(bl, oracle, M, N, K, seed, kind="laplace_channel", w_mean=0.001, full=True):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W, x = _case(M, N, K, seed, kind, w_mean)
     packed, a_g, beta = oracle.pack_bitnet(W.numpy())
     beta32 = np.float32(beta)
@@ -98,7 +98,7 @@ def test_w1a8_1p3b_sampled(bl, oracle, M, N, K):
 
 def test_w1a8_constant_and_alternating_tokens(bl, oracle):
     M, N, K = 20, 384, 256
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     x = synthetic.make_x("gauss_plain", M, K, 3)
     x[0] = 2.5                                     # constant token: gamma = 0
     x[1] = torch.tensor([1.0, -1.0] * (K // 2))    # alternating: codes +-127
@@ -119,7 +119,7 @@ def test_w1a8_constant_and_alternating_tokens(bl, oracle):
 
 def test_w1a8_unit_codes_give_popcount(bl):
     # with the quantisation bypassed and every code 1: acc_j = #pos - #neg
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     for M in (3, 150):
         N, K = 300, 512
         W = synthetic.weights(N, K, 8).cuda()
@@ -135,7 +135,7 @@ def test_w1a8_unit_codes_give_popcount(bl):
 
 def test_w1a8_guard_bands_and_error_word(bl, oracle):
     M, N, K = 140, 300, 384
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W, x = _case(M, N, K, 6)
     packed, _, beta = oracle.pack_bitnet(W.numpy())
     dp = torch.from_numpy(packed.view(np.int32)).cuda()
@@ -149,7 +149,7 @@ def test_w1a8_guard_bands_and_error_word(bl, oracle):
 
 def test_w1a8_end_to_end_pack_then_forward(bl, oracle):
     M, N, K = 200, 512, 1024
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W, x = _case(M, N, K, 12)
     packed_ref, _, beta_ref = oracle.pack_bitnet(W.numpy())
     gp, ga, gb = bl.bin_pack(W.cuda(), bl.BL_PACK_BITNET)

@@ -41,7 +41,7 @@ def _check_codes(oracle, xb, mode, xq_gpu, gamma_gpu):
 
 
 def _run(bl, oracle, M, N, K, seed, mode, ternary, full=True, x=None):
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     W = synthetic.weights(N, K, seed, mean=0.001)
     if x is None:
         x = synthetic.laplace_channel_activations(M, K, seed)
@@ -101,7 +101,7 @@ def test_per_tensor_gamma_differs_from_per_token(bl, oracle):
     """One token is a single spike, whose LN peak sqrt(K - 1) is the largest
     any token can have: it sets the shared gamma, so no other token reaches
     code 127 (under a per-token gamma every token does)."""
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     M, K = 4, 512
     x = synthetic.laplace_channel_activations(M, K, 3)
     x[1] = 0.0
@@ -129,7 +129,7 @@ def test_constant_rows_give_zero(bl, mode):
 
 def test_no_quant_flag_matches_plain_entry(bl):
     """Without a quantiser flag bitlinear_w1a8_ex is bitlinear_w1a8 / w158a8."""
-    from bit_linear_layers_b200 import synthetic
+    import synthetic
     M, N, K = 37, 300, 512
     x = synthetic.laplace_channel_activations(M, K, 9).cuda()
     packed = torch.randint(-2**31, 2**31 - 1, (N, K // 32), dtype=torch.int32, device="cuda")

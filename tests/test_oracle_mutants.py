@@ -76,6 +76,8 @@ MUTANTS = [
     ("ternary_acc_sign_ignored",
      "acc += (int64_t)ternary_value(packed, K, j, k) * (int64_t)xq[m * K + k];",
      "acc += (int64_t)(ternary_value(packed, K, j, k) != 0) * (int64_t)xq[m * K + k];"),
+    ("ternary_sample_index_swapped", "acc[i] = w158a8_acc_one(xq, packed, K, ms[i], js[i]);",
+     "acc[i] = w158a8_acc_one(xq, packed, K, js[i] % 5, ms[i]);"),
     # straight-through backward
     ("backward_dx_without_alpha", "s += bf16_value(dy[m * N + j]) * (double)alpha[j] * (double)packed_sign(packed, K, j, k);",
      "s += bf16_value(dy[m * N + j]) * (double)packed_sign(packed, K, j, k);"),

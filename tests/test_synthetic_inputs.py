@@ -7,7 +7,7 @@ import math
 import numpy as np
 import torch
 
-from bit_linear_layers_b200 import synthetic
+import synthetic
 
 
 def test_deterministic_per_seed_and_distinct_across_seeds():
