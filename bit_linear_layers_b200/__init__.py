@@ -234,9 +234,10 @@ class W1A16Stack:
 
     `levels` is a list of (x, linears), x a bf16 [K] (or [1, K]) device tensor
     and linears a list of (packed, alpha, y) with y a bf16 [N] (or [1, N])
-    tensor the call writes. A level may read any y of an earlier level. The
-    descriptor arrays are built once; run() enqueues the whole stack on the
-    current stream."""
+    tensor the call writes. Every y is its own buffer; a level's x is either
+    exactly the y of a linear of an earlier level or a buffer no linear
+    writes. The descriptor arrays are built once; run() enqueues the whole
+    stack on the current stream."""
 
     def __init__(self, levels, *, ws=None):
         jobs, lvls = [], []
@@ -260,7 +261,8 @@ class W1A16Stack:
         self._jobs = (StackJob * max(len(jobs), 1))(*jobs)
         self.num_levels, self.num_jobs = len(lvls), len(jobs)
         self.device = dev
-        self.ws, self.ws_bytes = _workspace(BL_OP_W1A16_STACK, 0, 0, 0, dev, ws)
+        total_n = sum(j.N for j in jobs)
+        self.ws, self.ws_bytes = _workspace(BL_OP_W1A16_STACK, 0, total_n, 0, dev, ws)
 
     def run(self):
         rc = lib.bin_linear_w1a16_stack(ctypes.byref(self._levels), self.num_levels, ctypes.byref(self._jobs),

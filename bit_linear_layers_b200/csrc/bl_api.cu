@@ -6,9 +6,12 @@
 // device code). Nothing here allocates memory.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "bitlinear.h"
 #include "bl_backward.cuh"
@@ -17,7 +20,7 @@
 #include "bl_gemv.cuh"
 #include "bl_gemv_lut.cuh"
 #include "bl_gemv_mma.cuh"
-#include "bl_gemv_stack.cuh"
+#include "bl_gemv_stream.cuh"
 #include "bl_lnquant.cuh"
 #include "bl_pack.cuh"
 #include "bl_xnor.cuh"
@@ -42,7 +45,7 @@ struct DeviceState {
   // can be resident at once: clusters must fit inside a GPC, so this is
   // below num_sms / S (on B200: 74 / 33 / 15)
   int cluster_cap[9] = {};
-  // clusters of 8 stacked-decode CTAs that can be resident at once
+  // clusters of 8 layer-stack decode CTAs that can be resident at once
   int stack_clusters = 0;
 };
 DeviceState g_devices[kMaxDevices];
@@ -86,7 +89,7 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<2>, 2 * kLutPageBytes) &&
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
               set_ts_smem<0>() && set_ts_smem<1>() && set_ts_smem<2>() &&
-              set_smem(gemv_w1a16_stack_kernel, kStackPages * kLutPageBytes) &&
+              set_smem(gemv_w1a16_stream_kernel, kStrSmemBytes) &&
               set_smem(gemm_ss_ste_kernel, kSsSmemBytes) &&
               set_smem(gemv_w1a16_mma_kernel<8, 16>, mma_smem_bytes(8, 16)) &&
               set_smem(gemv_w1a16_mma_kernel<16, 16>, mma_smem_bytes(16, 16)) &&
@@ -95,18 +98,18 @@ int device_setup(int* num_sms) {
     if (!ok) cudaGetLastError();
     {
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(kStackCluster, 1, 1);
-      cfg.blockDim = dim3(kLutThreads, 1, 1);
-      cfg.dynamicSmemBytes = kStackPages * kLutPageBytes;
+      cfg.gridDim = dim3(kStrCluster, 1, 1);
+      cfg.blockDim = dim3(kStrThreads + 32, 1, 1);
+      cfg.dynamicSmemBytes = kStrSmemBytes;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = kStackCluster;
+      attr[0].val.clusterDim.x = kStrCluster;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, gemv_w1a16_stack_kernel, &cfg) != cudaSuccess || n <= 0) {
+      if (cudaOccupancyMaxActiveClusters(&n, gemv_w1a16_stream_kernel, &cfg) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = 0;  // the stacked decode then reports BL_ERR_CUDA
       }
@@ -474,7 +477,7 @@ size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case BL_OP_W1A8_EX:
       return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double)) +
              align256(size_t(M) * sizeof(LnTokenStats)) + 256;
-    case BL_OP_W1A16_STACK: return kStackMaxLevels * sizeof(uint32_t);
+    case BL_OP_W1A16_STACK: return 256 + align256(size_t(N) * sizeof(uint32_t));
     case BL_OP_W1A16_BACKWARD: {
       const size_t Mp = size_t(cdiv(M, kSsUnit) * kSsUnit);
       return align256(size_t(M) * size_t(N) * 4) + align256(size_t(K) * size_t(N) / 4) +
@@ -600,78 +603,141 @@ int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const b
                            int num_jobs, void* ws, size_t ws_bytes, void* stream) {
   if (num_levels < 0 || num_jobs < 0) return BL_ERR_INVALID_ARG;
   if (num_levels == 0) return BL_OK;
-  if (!levels || !jobs || !ws || !aligned16(ws) || ws_bytes < bl_workspace_bytes(BL_OP_W1A16_STACK, 0, 0, 0))
-    return BL_ERR_INVALID_ARG;
+  if (!levels || !jobs || !ws || !aligned16(ws)) return BL_ERR_INVALID_ARG;
+  // level of every linear; the linears' outputs as byte ranges
+  std::vector<int> level_of(static_cast<size_t>(num_jobs), -1);
+  std::vector<std::pair<uintptr_t, int>> outs;  // (start, linear), sorted below
   for (int i = 0; i < num_levels; ++i) {
     const bl_stack_level& lv = levels[i];
     if (!lv.x || !aligned16(lv.x) || lv.num_jobs < 1 || lv.first_job < 0 ||
-        int64_t(lv.first_job) + lv.num_jobs > num_jobs || lv.num_jobs > kStackMaxJobs)
+        int64_t(lv.first_job) + lv.num_jobs > num_jobs || lv.num_jobs > kStrMaxJobs)
       return BL_ERR_INVALID_ARG;
-    if (lv.K < 256 || lv.K > 32 * kStackCluster * 16 * kStackPages || lv.K % 256 != 0) return BL_ERR_UNSUPPORTED;
+    if (lv.K < 256 || lv.K > 32 * kStrCluster * 48 || lv.K % 256 != 0) return BL_ERR_UNSUPPORTED;
     for (int j = lv.first_job; j < lv.first_job + lv.num_jobs; ++j) {
       const bl_stack_job& jb = jobs[j];
-      if (!jb.packed || !jb.alpha || !jb.y || jb.N < 1) return BL_ERR_INVALID_ARG;
+      if (level_of[size_t(j)] != -1) return BL_ERR_INVALID_ARG;  // a linear listed by two levels
+      if (!jb.packed || !jb.alpha || !jb.y || jb.N < 1 || !aligned16(jb.packed)) return BL_ERR_INVALID_ARG;
       if (jb.N > kMaxDim || jb.N * lv.K >= kMaxProduct) return BL_ERR_UNSUPPORTED;
+      level_of[size_t(j)] = i;
+      outs.emplace_back(reinterpret_cast<uintptr_t>(jb.y), j);
     }
   }
+  // every linear writes its own buffer
+  std::sort(outs.begin(), outs.end());
+  for (size_t t = 1; t < outs.size(); ++t)
+    if (outs[t].first < outs[t - 1].first + 2 * uintptr_t(jobs[outs[t - 1].second].N)) return BL_ERR_INVALID_ARG;
+  // the input of each level: a buffer written by no linear of the call, or
+  // exactly the output of one linear of an earlier level
+  std::vector<int> src(static_cast<size_t>(num_levels), -1);
+  int64_t total_n = 0;
+  for (int i = 0; i < num_levels; ++i) {
+    const uintptr_t x0 = reinterpret_cast<uintptr_t>(levels[i].x), x1 = x0 + 2 * uintptr_t(levels[i].K);
+    auto it = std::upper_bound(outs.begin(), outs.end(), std::make_pair(x1, -1));
+    if (it != outs.begin()) {
+      const auto& o = *(it - 1);  // the last output starting before x ends
+      const uintptr_t o1 = o.first + 2 * uintptr_t(jobs[o.second].N);
+      if (o1 > x0) {  // overlaps
+        if (o.first != x0 || jobs[o.second].N != levels[i].K || level_of[size_t(o.second)] >= i)
+          return BL_ERR_INVALID_ARG;
+        src[size_t(i)] = o.second;
+      }
+    }
+  }
+  for (int j = 0; j < num_jobs; ++j) total_n += level_of[size_t(j)] >= 0 ? jobs[j].N : 0;
+  if (ws_bytes < bl_workspace_bytes(BL_OP_W1A16_STACK, 0, total_n, 0)) return BL_ERR_INVALID_ARG;
   int sms = 0;
   int rc = device_setup(&sms);
   if (rc != BL_OK) return rc;
   const int G = stack_cluster_capacity();
   if (G < 1) return BL_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint32_t* done = static_cast<uint32_t*>(ws);
-  // one launch per run of at most kStackMaxLevels levels / kStackMaxJobs linears
-  static thread_local StackParams P;  // 12 KB: too large for the stack of every caller
+
+  // Launches of at most kStrMaxLevels levels and kStrMaxJobs linears. An
+  // output read by a later level of the same launch gets a tagged copy in
+  // the workspace; the copies are zero-filled once, before the first launch.
+  std::vector<int> launch_of(static_cast<size_t>(num_levels));
+  {
+    int li = 0, nl = 0, nj = 0;
+    for (int i = 0; i < num_levels; ++i) {
+      if (nl == kStrMaxLevels || nj + levels[i].num_jobs > kStrMaxJobs) {
+        ++li;
+        nl = nj = 0;
+      }
+      launch_of[size_t(i)] = li;
+      ++nl;
+      nj += levels[i].num_jobs;
+    }
+  }
+  std::vector<int64_t> tag_off(static_cast<size_t>(num_jobs), -1);
+  int64_t tagged_words = 0;
+  for (int i = 0; i < num_levels; ++i) {
+    const int j = src[size_t(i)];
+    if (j >= 0 && launch_of[size_t(level_of[size_t(j)])] == launch_of[size_t(i)] && tag_off[size_t(j)] < 0) {
+      tag_off[size_t(j)] = tagged_words;
+      tagged_words += jobs[j].N;
+    }
+  }
+  // ws: the abort word (first 256 bytes), then the tagged outputs; only
+  // launches with tagged outputs wait on anything outside their clusters
+  uint32_t* abort_word = static_cast<uint32_t*>(ws);
+  uint32_t* tags = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 256);
+  if (tagged_words > 0 && cudaMemsetAsync(ws, 0, 256 + size_t(tagged_words) * 4, s) != cudaSuccess) {
+    cudaGetLastError();
+    return BL_ERR_CUDA;
+  }
+  static thread_local StrParams P;  // ~29 KB: too large for the stack of every caller
   int i = 0;
   while (i < num_levels) {
     std::memset(&P, 0, sizeof P);
+    const int li = launch_of[size_t(i)];
     int nl = 0, nj = 0;
-    int64_t max_blocks = 0;
-    while (i < num_levels && nl < kStackMaxLevels && nj + levels[i].num_jobs <= kStackMaxJobs) {
+    int64_t max_chunks = 0;
+    for (; i < num_levels && launch_of[size_t(i)] == li; ++i) {
       const bl_stack_level& lv = levels[i];
-      StackLevel& d = P.lv[nl];
-      d.x = lv.x;
+      StrLevel& d = P.lv[nl++];
+      const int j_src = src[size_t(i)];
+      if (j_src >= 0 && tag_off[size_t(j_src)] >= 0)
+        d.xt = tags + tag_off[size_t(j_src)];
+      else
+        d.x = lv.x;
       d.K = int(lv.K);
       d.job0 = nj;
       d.njobs = lv.num_jobs;
-      int64_t blocks = 0;
+      int64_t chunks = 0;
       for (int j = lv.first_job; j < lv.first_job + lv.num_jobs; ++j) {
-        StackJob& e = P.jb[nj++];
-        e.packed = jobs[j].packed;
+        StrJob& e = P.jobs[nj];
+        if (!make_map_2d(&P.maps[nj], jobs[j].packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(lv.K / 32),
+                         uint64_t(jobs[j].N), 16, kStrBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+          return BL_ERR_CUDA;
+        ++nj;
         e.alpha = jobs[j].alpha;
         e.y = jobs[j].y;
+        e.tagged = tag_off[size_t(j)] >= 0 ? tags + tag_off[size_t(j)] : nullptr;
         e.N = int(jobs[j].N);
-        e.block0 = int(blocks);
-        blocks += cdiv(jobs[j].N, kLutRowsPerCluster);
+        e.chunk0 = int(chunks);
+        chunks += cdiv(jobs[j].N, kStrChunk);
       }
-      if (blocks > kMaxDim) return BL_ERR_UNSUPPORTED;
-      d.nblocks = int(blocks);
-      if (blocks > max_blocks) max_blocks = blocks;
-      ++nl;
-      ++i;
+      if (chunks > kMaxDim / kStrChunk) return BL_ERR_UNSUPPORTED;
+      d.nchunks = int(chunks);
+      if (chunks > max_chunks) max_chunks = chunks;
     }
-    const int clusters = int(max_blocks < G ? max_blocks : G);
-    P.done = done;
     P.num_levels = nl;
-    P.total_ctas = clusters * kStackCluster;
-    if (cudaMemsetAsync(done, 0, size_t(nl) * sizeof(uint32_t), s) != cudaSuccess) {
-      cudaGetLastError();
-      return BL_ERR_CUDA;
-    }
+    P.num_jobs = nj;
+    P.abort = abort_word;
+    const int clusters = int(max_chunks < G ? max_chunks : G);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kStackCluster, static_cast<unsigned>(clusters), 1);
-    cfg.blockDim = dim3(kLutThreads, 1, 1);
-    cfg.dynamicSmemBytes = kStackPages * kLutPageBytes;
+    cfg.gridDim = dim3(kStrCluster, static_cast<unsigned>(clusters), 1);
+    cfg.blockDim = dim3(kStrThreads + 32, 1, 1);
+    cfg.dynamicSmemBytes = kStrSmemBytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kStackCluster;
+    attr[0].val.clusterDim.x = kStrCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemv_w1a16_stack_kernel, P) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, gemv_w1a16_stream_kernel, P) != cudaSuccess) {
       cudaGetLastError();
       return BL_ERR_CUDA;
     }

@@ -36,6 +36,7 @@ enum : int {
   kWhereSsMma = 9,
   kWhereSsEpilogue = 10,
   kWhereMmaInbox = 11,  // the few-token warp-MMA GEMV
+  kWhereStackRing = 12, // a layer-stack weight slot
 };
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.

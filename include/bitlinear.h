@@ -67,7 +67,7 @@ extern "C" {
 #define BL_OP_PACK_TERNARY 4
 #define BL_OP_W158A8 5
 #define BL_OP_W1A8_EX 6 /* bitlinear_w1a8_ex with a per-tensor quantiser */
-#define BL_OP_W1A16_STACK 7 /* bin_linear_w1a16_stack (M, N, K ignored) */
+#define BL_OP_W1A16_STACK 7 /* bin_linear_w1a16_stack (N = total outputs; M, K ignored) */
 #define BL_OP_W1A16_BACKWARD 8 /* bin_linear_w1a16_backward */
 
 /* Library ABI version (this header: 1). */
@@ -163,24 +163,28 @@ int bin_linear_w1a16_backward(const uint16_t* x, const uint32_t* packed, const f
 /*
  * bin_linear_w1a16_stack -- single-token decode through a stack of FBI-linear
  * layers in one persistent launch (the same y = bf16(alpha * sum s x) as
- * bin_linear_w1a16 at M = 1, for every linear of the stack, in order).
+ * bin_linear_w1a16 at M = 1, for every linear of the stack).
  *
  * The stack is a sequence of levels. Level i reads one input vector
  * levels[i].x (K bf16) and runs the linears jobs[first_job .. first_job +
- * num_jobs), each writing its own y (N bf16). A level starts only after every
- * linear of the levels before it has written its output, so levels[i].x may
- * be any y of an earlier level (or a buffer written before the call); two
- * linears of one level must not write a buffer that level reads.
- * Limits: K a multiple of 256 and at most 12288; 1 <= N < 2^31; x 16-byte
- * aligned. Results are bit-identical to bin_linear_w1a16 whenever that call
- * splits K eight ways (K/32 words a multiple of 8, 128..384 of them, e.g.
- * K = 4096 and 11008).
- * The call enqueues one zero-fill of ws and one kernel per 128 levels (or
- * per 256 linears) on `stream`. ws: bl_workspace_bytes(BL_OP_W1A16_STACK,
- * 0, 0, 0) bytes of device memory, 16-byte aligned, not shared with a call
- * still running. The kernel needs every one of its CTAs resident at once
- * (one per SM in clusters of 8): if the GPU cannot host them all it records
- * BL_ERR_TIMEOUT (bl_device_error) instead of waiting forever.
+ * num_jobs), each writing its own y (N bf16). levels[i].x is either exactly
+ * the y of one linear of an earlier level (same pointer, N == K) or a buffer
+ * written before the call that no linear of the stack writes; every linear's
+ * y is a buffer of its own (no two overlap). Other stacks are rejected with
+ * BL_ERR_INVALID_ARG. A level starts as soon as its own input is complete.
+ * Limits: K a multiple of 256, 256 <= K <= 12288; 1 <= N < 2^31; x and
+ * packed 16-byte aligned. Results are bit-identical to bin_linear_w1a16
+ * whenever that call splits K eight ways (K/32 words a multiple of 8, 128..384
+ * of them, e.g. K = 4096 and 11008).
+ * The weights of the levels ahead stream into shared memory while a level
+ * waits for its input. The call enqueues at most one zero-fill of ws and one
+ * kernel per 96 levels (or per 144 linears) on `stream`. ws:
+ * bl_workspace_bytes(BL_OP_W1A16_STACK, 0, total_N, 0) bytes of device
+ * memory, 16-byte aligned, not shared with a call still running, where
+ * total_N is the sum of N over the stack's linears. The kernel needs every
+ * one of its CTAs resident at once (one per SM in clusters of 8): if the GPU
+ * cannot host them all it records BL_ERR_TIMEOUT (bl_device_error) instead of
+ * waiting forever.
  */
 typedef struct bl_stack_job {
   const uint32_t* packed; /* [N x K/32] */

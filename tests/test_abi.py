@@ -89,19 +89,45 @@ def test_null_and_misaligned_pointers_rejected():
 
 def test_stack_validation_without_device_work():
     import bit_linear_layers_b200 as bl
-    job = bl.StackJob(FAKE.value, FAKE.value, FAKE.value, 256)
-    ws = bl.workspace_bytes(bl.BL_OP_W1A16_STACK, 0, 0, 0)
-    assert ws >= 128 * 4
+    N, K = 256, 4096
+    Y0, Y1, X = 0x100000, 0x200000, 0x300000  # never dereferenced: every check below is on the host
+    job = bl.StackJob(FAKE.value, FAKE.value, Y0, N)
+    ws = bl.workspace_bytes(bl.BL_OP_W1A16_STACK, 0, N, 0)
+    assert ws >= 256 + 4 * N
 
-    def call(K, first=0, num=1, n_levels=1, ws_bytes=ws, x=FAKE.value):
+    def call(K, first=0, num=1, n_levels=1, ws_bytes=ws, x=X):
         lv = bl.StackLevel(x, K, first, num)
         return bl.lib.bin_linear_w1a16_stack(ctypes.byref(lv), n_levels, ctypes.byref(job), 1, FAKE, ws_bytes, None)
 
     assert call(4096, n_levels=0) == 0              # empty stack: nothing to do
-    assert call(4000) == -2 and call(12544) == -2   # K % 256, more than three table pages
+    assert call(4000) == -2 and call(12544) == -2   # K % 256, more than 48 words per slice
     assert call(4096, first=1) == -1 and call(4096, num=0) == -1
     assert call(4096, ws_bytes=8) == -1
     assert call(4096, x=ODD.value) == -1
+    assert call(4096, x=Y0) == -1                   # reads the output of its own level
+    assert call(4096, x=Y0 + 2 * N - 2) == -1       # overlaps it
+    assert call(4096) == bl.BL_ERR_NO_DEVICE        # valid: stops only at the device
+
+    def stack(specs, jobs, ws_bytes=1 << 20):
+        """specs: (x, K, first, num) per level; jobs: (y, N)."""
+        lvs = (bl.StackLevel * len(specs))(*[bl.StackLevel(*sp) for sp in specs])
+        jbs = (bl.StackJob * len(jobs))(*[bl.StackJob(FAKE.value, FAKE.value, y, n) for y, n in jobs])
+        return bl.lib.bin_linear_w1a16_stack(lvs, len(specs), jbs, len(jobs), FAKE, ws_bytes, None)
+
+    # level 1 reads level 0's output exactly: valid
+    assert stack([(X, K, 0, 1), (Y0, K, 1, 1)], [(Y0, K), (Y1, 128)]) == bl.BL_ERR_NO_DEVICE
+    # ... but not with a different length, nor part of it
+    assert stack([(X, K, 0, 1), (Y0, 2048, 1, 1)], [(Y0, K), (Y1, 128)]) == -1
+    assert stack([(X, K, 0, 1), (Y0 + 256, K, 1, 1)], [(Y0, 2 * K), (Y1, 128)]) == -1
+    # an input written by a later level
+    assert stack([(Y1, K, 0, 1), (X, K, 1, 1)], [(Y0, K), (Y1, K)]) == -1
+    # two linears writing overlapping outputs
+    assert stack([(X, K, 0, 2)], [(Y0, K), (Y0 + 2 * K - 2, K)]) == -1
+    assert stack([(X, K, 0, 1), (Y0, K, 1, 1)], [(Y0, K), (Y0, K)]) == -1
+    # a linear listed by two levels
+    assert stack([(X, K, 0, 1), (Y0, K, 0, 1)], [(Y0, K)]) == -1
+    # the workspace must hold a tagged word per output
+    assert stack([(X, K, 0, 1), (Y0, K, 1, 1)], [(Y0, K), (Y1, 128)], ws_bytes=256 + 4 * K) == -1
 
 
 def test_backward_validation_without_device_work():

@@ -7,7 +7,7 @@ layers in one persistent launch) on the GPU.
   level, and inputs produced by earlier levels;
 * bit-identical to bin_linear_w1a16 called layer by layer where that call
   also splits K eight ways (K = 4096 and 11008, the 7B shapes);
-* stacks longer than one launch (more than 128 levels or 256 linears);
+* stacks longer than one launch (more than 96 levels or 144 linears);
 * the argument checks."""
 import ctypes
 
@@ -133,7 +133,7 @@ def test_stack_longer_than_one_launch(bl, oracle):
 
 
 def test_stack_many_linears_per_launch(bl, oracle):
-    # 300 linears over 3 levels (more than 256 linears: split between launches)
+    # 300 linears over 3 levels (more than 144 linears: split between launches)
     import synthetic
     K = 256
     dp, da, packed, alpha = _linear(oracle, 64, K, 90)
@@ -153,7 +153,7 @@ def test_stack_argument_checks(bl):
     p = torch.zeros((N, K // 32), dtype=torch.int32, device="cuda")
     a = torch.zeros(N, dtype=torch.float32, device="cuda")
     y = torch.zeros(N, dtype=torch.bfloat16, device="cuda")
-    ws = torch.zeros(bl.workspace_bytes(bl.BL_OP_W1A16_STACK, 0, 0, 0), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(bl.workspace_bytes(bl.BL_OP_W1A16_STACK, 0, N, 0), dtype=torch.uint8, device="cuda")
     job = bl.StackJob(p.data_ptr(), a.data_ptr(), y.data_ptr(), N)
 
     def call(K_, first=0, num=1, ws_bytes=ws.numel(), xp=x.data_ptr()):
@@ -163,7 +163,7 @@ def test_stack_argument_checks(bl):
 
     assert call(4096) == 0
     assert call(4000) == bl.BL_ERR_UNSUPPORTED     # not a multiple of 256
-    assert call(12544) == bl.BL_ERR_UNSUPPORTED    # beyond three table pages
+    assert call(12544) == bl.BL_ERR_UNSUPPORTED    # more than 48 words per slice
     assert call(4096, first=1) == bl.BL_ERR_INVALID_ARG
     assert call(4096, num=0) == bl.BL_ERR_INVALID_ARG
     assert call(4096, ws_bytes=4) == bl.BL_ERR_INVALID_ARG
