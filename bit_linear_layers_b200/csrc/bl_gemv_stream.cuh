@@ -168,8 +168,9 @@ __device__ __forceinline__ void str_seek(const StrJob* jobs, const StrLevel& lv,
 // cluster cid's run of chunks of level lv (empty when the level has fewer chunks than clusters)
 __device__ __forceinline__ StrRun str_run(const StrJob* jobs, const StrLevel& lv, int cid, int G) {
   StrRun r;
-  r.cur = static_cast<int>((static_cast<int64_t>(lv.nchunks) * cid) / G);
-  r.end = static_cast<int>((static_cast<int64_t>(lv.nchunks) * (cid + 1)) / G);
+  // nchunks < 2^27 and G <= 32: the products fit 32 bits
+  r.cur = static_cast<int>((static_cast<uint32_t>(lv.nchunks) * static_cast<uint32_t>(cid)) / static_cast<uint32_t>(G));
+  r.end = static_cast<int>((static_cast<uint32_t>(lv.nchunks) * static_cast<uint32_t>(cid + 1)) / static_cast<uint32_t>(G));
   r.j = lv.job0;
   r.jlast = lv.job0 + lv.njobs - 1;
   r.jbeg = 0;
