@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--probe-int8", action="store_true",
+                    help="measure the dense int8 tensor throughput of this GPU (torch._int_mm, 8192^3) and exit")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the other workloads and the 7B measurement that ride along at N=1")
     a = ap.parse_args()
@@ -528,6 +530,87 @@ class W1A8(Workload):
             self.o.w1a8(x, p, beta, K)
 
 
+class W1A8Single(Workload):
+    """BitNet BitLinear, one small layer: M=4 tokens, K=N=256, seed 0. The
+    whole forward (LN, per-token absmax int8 quantisation, +-1 products,
+    beta*gamma/128 rescale) is one fused launch; the problem is latency-bound
+    (14 KB of operands), so the roofline fraction is tiny by construction."""
+    name = "w1a8_single"
+    M, K, N = 4, 256, 256
+    metric = "BitLinear W1A8 single layer tokens/s (M=4, K=N=256, LN + absmax quant + int8 products + rescale)"
+    unit, scale, bound = "tok/s", 1.0, "hbm"
+    dtype = "s8"
+    kernel = "bitlinear_small_kernel<4,false> (one fused launch per call)"
+    sources = [CSRC + "bl_gemv.cuh", CSRC + "bl_lnquant.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    roof_unit = "GB/s"
+    rotate = 18000  # 14 KB per copy: 250 MB, about twice the L2
+
+    def __init__(self):
+        M, K, N = self.M, self.K, self.N
+        self.bytes_per_call = N * K // 8 + 2 * M * K + 4 * M * N + 4
+        self.config = {"workload": "BitNet BitLinear W1A8 single layer, M=4 tokens, K=N=256, seed 0",
+                       "M": M, "K": K, "N": N,
+                       "l2": f"inputs larger than L2: {self.rotate} distinct copies of weights, activations and "
+                             f"outputs ({self.rotate * self.bytes_per_call / 1e6:.0f} MB) rotated step to step",
+                       "launch": "one fused kernel per call"}
+
+    def units_per_step(self):
+        return float(self.M)  # tokens
+
+    def achieved(self, per_step_s):
+        return self.bytes_per_call / per_step_s / 1e9  # bytes the call must move
+
+    def peak(self, peaks, timed_s):
+        return peaks["hbm_gbs"], "hbm_gbs"
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        import synthetic
+        self.bl = bl
+        M, K, N = self.M, self.K, self.N
+        # copy 0 is the seeded workload; the others are further seeded draws made on the device
+        W = synthetic.weights(N * self.rotate, K, seed=replica_seed(0, 1, rank), device=dev)
+        W[:N] = synthetic.weights(N, K, seed=0).to(dev)
+        X = synthetic.activations(M * self.rotate, K, seed=replica_seed(0, 1, rank), device=dev)
+        X[:M] = synthetic.activations(M, K, seed=0).to(dev)
+        self.ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W1A8, M, N, K), dtype=torch.uint8, device=dev)
+        self.copies = []
+        for i in range(self.rotate):
+            p, _, b = bl.bin_pack(W[i * N:(i + 1) * N], bl.BL_PACK_BITNET)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            self.copies.append((X[i * M:(i + 1) * M], p, b, y))
+        del W
+        self.xh = [self.copies[i][0].cpu().pin_memory() for i in range(16)]
+        self.yh = [torch.empty((M, N), dtype=torch.float32).pin_memory() for _ in range(16)]
+        self.xd = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.yd = torch.empty((M, N), dtype=torch.float32, device=dev)
+        self.h2d, self.d2h = 2 * M * K, 4 * M * N
+
+    def step(self, i):
+        x, p, b, y = self.copies[i % self.rotate]
+        self.bl.bitlinear_w1a8(x, p, b, out=y, ws=self.ws)
+
+    def e2e_step(self, i):
+        _, p, b, _ = self.copies[i % self.rotate]
+        self.xd.copy_(self.xh[i % 16], non_blocking=True)
+        self.bl.bitlinear_w1a8(self.xd, p, b, out=self.yd, ws=self.ws)
+        self.yh[i % 16].copy_(self.yd, non_blocking=True)
+
+    def oracle_setup(self):
+        import oracle as oracle_pkg
+        import synthetic
+        self.o = oracle_pkg.get()
+        W = synthetic.weights(self.N, self.K, seed=0).numpy()
+        self.op, _, self.obeta = self.o.pack_bitnet(W)
+        self.ox = synthetic.bf16_bits(synthetic.activations(self.M, self.K, seed=0))
+        self.oracle_sample = "the whole M=4, K=N=256 layer per call (single-threaded C oracle, fp64/int64)"
+        return float(self.M)
+
+    def oracle_call(self):
+        self.o.w1a8(self.ox, self.op, self.obeta, self.K)
+
+
 class W158A8(W1A8):
     """BitNet b1.58: the W1A8 workload with ternary weights (RoundClip of
     W / mean|W|, two bit planes)."""
@@ -721,7 +804,7 @@ class W1A1(Workload):
             self.o.w1a1(a, b, K)
 
 
-WORKLOADS = {w.name: w for w in (Decode, Prefill, Backward, W1A8, W158A8, W1A8Tensor, W1A1)}
+WORKLOADS = {w.name: w for w in (Decode, Prefill, Backward, W1A8, W1A8Single, W158A8, W1A8Tensor, W1A1)}
 
 
 # ----------------------------------------------------------------------------- ours
@@ -836,7 +919,7 @@ def summarize(wl, ms, ms_e2e, steps, world, peaks, peak_kind):
     timed_s = ms * 1e-3
     peak, peak_key = wl.peak(peaks, timed_s)
     achieved = wl.achieved(per_step_s)
-    roof = {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": wl.unit,
+    roof = {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": getattr(wl, "roof_unit", wl.unit),
             "frac": achieved / peak, "traffic": wl.traffic(), "kernel": wl.kernel,
             "peak_source": peak_key if peak_key.startswith("derived")
             else (f"{peak_kind}: MEASURED_PEAKS.json {peak_key}" if peak_kind == "measured" else f"fallback ({peak_key})")}
@@ -910,38 +993,39 @@ def secondary_llama7b(dev, peaks):
                                    "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                    "launches_per_step": 224}
         del gph
-        if B == 1:
-            # the same chain as one stacked call: 128 levels (q,k,v | o | gate,up | down per
-            # layer), every linear writing a buffer of its own
-            levels = []
-            cur = x.reshape(-1)
-            for mats in layers:
-                lq, lk, lv, lo, lh = (torch.empty(4096, dtype=torch.bfloat16, device=dev) for _ in range(5))
-                lg, lu = (torch.empty(11008, dtype=torch.bfloat16, device=dev) for _ in range(2))
-                levels.append((cur, [(mats[0][0], mats[0][1], lq), (mats[1][0], mats[1][1], lk),
-                                     (mats[2][0], mats[2][1], lv)]))
-                levels.append((lv, [(mats[3][0], mats[3][1], lo)]))
-                levels.append((lo, [(mats[4][0], mats[4][1], lg), (mats[5][0], mats[5][1], lu)]))
-                levels.append((lu, [(mats[6][0], mats[6][1], lh)]))
-                cur = lh
-            stack = bl.W1A16Stack(levels)
-            for _ in range(3):
-                stack.run()
-            torch.cuda.synchronize()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(reps):
-                stack.run()
-            e1.record()
-            torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1) / reps
-            res["decode_batch1_stack"] = {
-                "ms_per_token_step": ms, "tok_s": 1.0 / (ms * 1e-3),
-                "packed_GB_per_s": packed_bytes / (ms * 1e-3) / 1e9,
-                "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                "launches_per_step": 2, "call": "bin_linear_w1a16_stack (one zero-fill of the tagged outputs + "
-                                                 "two persistent kernels)"}
+        # the same chain as one stacked call: 128 levels (q,k,v | o | gate,up | down per
+        # layer), every linear writing a buffer of its own
+        levels = []
+        cur = x.reshape(-1) if B == 1 else x
+        shp = (lambda n: (n,)) if B == 1 else (lambda n: (B, n))
+        for mats in layers:
+            lq, lk, lv, lo, lh = (torch.empty(shp(4096), dtype=torch.bfloat16, device=dev) for _ in range(5))
+            lg, lu = (torch.empty(shp(11008), dtype=torch.bfloat16, device=dev) for _ in range(2))
+            levels.append((cur, [(mats[0][0], mats[0][1], lq), (mats[1][0], mats[1][1], lk),
+                                 (mats[2][0], mats[2][1], lv)]))
+            levels.append((lv, [(mats[3][0], mats[3][1], lo)]))
+            levels.append((lo, [(mats[4][0], mats[4][1], lg), (mats[5][0], mats[5][1], lu)]))
+            levels.append((lu, [(mats[6][0], mats[6][1], lh)]))
+            cur = lh
+        stack = bl.W1A16Stack(levels)
+        for _ in range(3):
+            stack.run()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            stack.run()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[f"decode_batch{B}_stack"] = {
+            "ms_per_token_step": ms, "tok_s": B / (ms * 1e-3),
+            "packed_GB_per_s": packed_bytes / (ms * 1e-3) / 1e9,
+            "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "launches_per_step": 3, "call": "bin_linear_w1a16_stack_batch (one zero-fill of the tagged outputs + "
+                                             "two persistent kernels)"}
+        del stack, levels
     # prefill: 4096 tokens through every linear (not chained: fixed inputs)
     T = 4096
     x4 = synthetic.activations(T, 4096, seed=78, device=dev)
@@ -991,9 +1075,83 @@ def secondary(args, dev, peaks, peak_kind):
         gc.collect()
         torch.cuda.empty_cache()
     out["pack"] = secondary_pack(dev, peaks)
+    out["few_tokens"] = secondary_few_tokens(dev, peaks)
     out["decode_l2_warm"] = secondary_decode_warm(dev)
     out["llama7b_linear"] = secondary_llama7b(dev, peaks)
     return out
+
+
+def secondary_few_tokens(dev, peaks):
+    """The few-token paths at decode shapes, each timed as a graph of launches
+    over rotating copies (more than L2): W1A16 at 2..16 tokens on 4096x4096
+    (the 7B attention projection) and W1A8 at 1..16 tokens on 2048->5632 (the
+    1.3B MLP up-projection); GB/s counts the bytes a call must move."""
+    import torch
+    import bit_linear_layers_b200 as bl
+    import synthetic
+    res = {"l2": "rotating copies larger than L2; one CUDA graph of 400 calls, CUDA events"}
+    calls = 400
+
+    def time_graph(fn, n):
+        st = torch.cuda.Stream(device=dev)
+        st.wait_stream(torch.cuda.current_stream(dev))
+        for i in range(8):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(g, stream=st):
+                for i in range(n):
+                    fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        ms = _median_ms(g.replay, reps=5)
+        del g
+        return ms / n
+
+    K = N = 4096
+    copies = 64  # 2 MB of signs each
+    packs = []
+    for i in range(copies):
+        W = synthetic.weights(N, K, seed=3000 + i, device=dev)
+        packs.append(bl.bin_pack(W, bl.BL_PACK_FBI))
+        del W
+    for M in (2, 4, 8, 16):
+        xs = [synthetic.activations(M, K, seed=3100 + i, device=dev) for i in range(copies)]
+        ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+
+        def fn(i, xs=xs, ys=ys):
+            j = i % copies
+            bl.bin_linear_w1a16(xs[j], *packs[j], out=ys[j], flags=bl.BL_FLAG_OVERLAP_PREVIOUS)
+
+        s_call = time_graph(fn, calls) * 1e-3
+        nbytes = N * K // 8 + 4 * N + 2 * M * K + 2 * M * N
+        res[f"w1a16_M{M}_4096x4096"] = {"us_per_call": s_call * 1e6, "GB_s": nbytes / s_call / 1e9,
+                                        "hbm_frac": nbytes / s_call / 1e9 / peaks["hbm_gbs"]}
+    del packs
+    K, N = 2048, 5632
+    copies = 96  # 1.4 MB of signs each
+    layers = []
+    for i in range(copies):
+        W = synthetic.weights(N, K, seed=3200 + i, mean=0.001, device=dev)
+        p, _, b = bl.bin_pack(W, bl.BL_PACK_BITNET)
+        layers.append((p, b))
+        del W
+    for M in (1, 4, 16):
+        xs = [synthetic.laplace_channel_activations(M, K, seed=3300 + i, device=dev) for i in range(copies)]
+        ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for _ in range(copies)]
+        ws = torch.empty(bl.workspace_bytes(bl.BL_OP_W1A8, M, N, K), dtype=torch.uint8, device=dev)
+
+        def fn(i, xs=xs, ys=ys, ws=ws):
+            j = i % copies
+            bl.bitlinear_w1a8(xs[j], *layers[j], out=ys[j], ws=ws)
+
+        s_call = time_graph(fn, calls) * 1e-3
+        nbytes = N * K // 8 + 2 * M * K + 4 * M * N
+        res[f"w1a8_M{M}_2048x5632"] = {"us_per_call": s_call * 1e6, "GB_s": nbytes / s_call / 1e9,
+                                       "hbm_frac": nbytes / s_call / 1e9 / peaks["hbm_gbs"],
+                                       "launches": 2}
+    return res
 
 
 def secondary_pack(dev, peaks):
@@ -1075,8 +1233,46 @@ def _median_ms(fn, reps=5):
 # ----------------------------------------------------------------------------- main
 
 
+def probe_int8(dev):
+    """Dense int8 GEMM throughput of a library kernel (torch._int_mm, s8 x s8
+    -> s32, M = N = K = 8192): best of 10 launches and the mean of a 2 s loop,
+    in TOP/s (2 MNK per product). A reference point for the W1A8 rooflines."""
+    import torch
+    n = 8192
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t().contiguous().t()
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize()
+    best = min(_median_ms(lambda: torch._int_mm(a, b), reps=1) for _ in range(10))
+    reps, t_end = 0, time.time() + 2.0
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    while time.time() < t_end:
+        for _ in range(20):
+            torch._int_mm(a, b)
+        reps += 20
+    e1.record()
+    torch.cuda.synchronize()
+    sustained = e0.elapsed_time(e1) / reps
+    ops = 2.0 * n ** 3
+    return {"probe": "torch._int_mm s8 x s8 -> s32, 8192^3", "burst_tops": ops / (best * 1e-3) / 1e12,
+            "sustained_tops": ops / (sustained * 1e-3) / 1e12, "best_ms": best, "sustained_ms": sustained,
+            "gpu": torch.cuda.get_device_name(dev)}
+
+
 def main():
     args = parse()
+    if args.probe_int8:
+        import torch
+        dev = torch.device("cuda", 0)
+        sampler = ClockSampler(0)
+        sampler.start()
+        res = probe_int8(dev)
+        res["clocks"] = sampler.stop()
+        print(json.dumps(res), flush=True)
+        return 0
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

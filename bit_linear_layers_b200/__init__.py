@@ -85,6 +85,7 @@ SIGNATURES = {
     "bitlinear_w1a8_noalloc": ([_p, _p, _p, _p, _i64, _i64, _i64, _p], _int),
     "bin_xnor_gemm": ([_p, _p, _p, _i64, _i64, _i64, _p], _int),
     "bin_linear_w1a16_stack": ([_p, _int, _p, _int, _p, _sz, _p], _int),
+    "bin_linear_w1a16_stack_batch": ([_p, _int, _p, _int, _i64, _p, _sz, _p], _int),
     "bin_linear_w1a16_backward": ([_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
     "bitlinear_w1a8_ex": ([_p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_uint, _p, _sz, _p, _p, _p, _p], _int),
     "bitlinear_w158a8": ([_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p], _int),
@@ -230,28 +231,32 @@ def bin_linear_w1a16_backward(x: torch.Tensor, packed: torch.Tensor, alpha: torc
 
 
 class W1A16Stack:
-    """A stack of single-token FBI-linear layers run by bin_linear_w1a16_stack.
+    """A stack of FBI-linear layers decoded by bin_linear_w1a16_stack(_batch).
 
-    `levels` is a list of (x, linears), x a bf16 [K] (or [1, K]) device tensor
-    and linears a list of (packed, alpha, y) with y a bf16 [N] (or [1, N])
-    tensor the call writes. Every y is its own buffer; a level's x is either
-    exactly the y of a linear of an earlier level or a buffer no linear
-    writes. The descriptor arrays are built once; run() enqueues the whole
-    stack on the current stream."""
+    `levels` is a list of (x, linears), x a bf16 [K] or [M, K] device tensor
+    (M tokens, 1 <= M <= 16, the same for every level) and linears a list of
+    (packed, alpha, y) with y a bf16 [N] or [M, N] tensor the call writes.
+    Every y is its own buffer; a level's x is either exactly the y of a
+    linear of an earlier level or a buffer no linear writes. The descriptor
+    arrays are built once; run() enqueues the whole stack on the current
+    stream."""
 
     def __init__(self, levels, *, ws=None):
         jobs, lvls = [], []
         self._keep = []
         dev = None
+        M = None
         for x, linears in levels:
             K = x.shape[-1]
-            if x.numel() != K:
-                raise ValueError("stack inputs are single vectors")
+            m = x.numel() // K
+            if x.numel() != m * K or (M is not None and m != M):
+                raise ValueError("stack inputs are [M, K] with the same M for every level")
+            M = m
             dev = x.device
             lvls.append(StackLevel(_dev_ptr(x, torch.bfloat16, "x"), K, len(jobs), len(linears)))
             for packed, alpha, y in linears:
                 N = packed.shape[0]
-                if y.numel() != N or packed.shape[1] * 32 != K:
+                if y.numel() != M * N or packed.shape[1] * 32 != K:
                     raise ValueError("linear shapes do not match the level input")
                 jobs.append(StackJob(_dev_ptr(packed, torch.int32, "packed"), _dev_ptr(alpha, torch.float32, "alpha"),
                                      _dev_ptr(y, torch.bfloat16, "y"), N))
@@ -260,15 +265,16 @@ class W1A16Stack:
         self._levels = (StackLevel * max(len(lvls), 1))(*lvls)
         self._jobs = (StackJob * max(len(jobs), 1))(*jobs)
         self.num_levels, self.num_jobs = len(lvls), len(jobs)
+        self.M = M or 1
         self.device = dev
         total_n = sum(j.N for j in jobs)
-        self.ws, self.ws_bytes = _workspace(BL_OP_W1A16_STACK, 0, total_n, 0, dev, ws)
+        self.ws, self.ws_bytes = _workspace(BL_OP_W1A16_STACK, self.M, total_n, 0, dev, ws)
 
     def run(self):
-        rc = lib.bin_linear_w1a16_stack(ctypes.byref(self._levels), self.num_levels, ctypes.byref(self._jobs),
-                                        self.num_jobs, _dev_ptr(self.ws, torch.uint8, "ws"), self.ws.numel(),
-                                        _stream(self.device))
-        _check("bin_linear_w1a16_stack", rc)
+        rc = lib.bin_linear_w1a16_stack_batch(ctypes.byref(self._levels), self.num_levels, ctypes.byref(self._jobs),
+                                              self.num_jobs, self.M, _dev_ptr(self.ws, torch.uint8, "ws"),
+                                              self.ws.numel(), _stream(self.device))
+        _check("bin_linear_w1a16_stack_batch", rc)
 
 
 def bitlinear_w1a8(x: torch.Tensor, packed: torch.Tensor, beta: torch.Tensor, *, out=None, ws=None):

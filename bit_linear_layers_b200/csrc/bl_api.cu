@@ -21,6 +21,7 @@
 #include "bl_gemv_lut.cuh"
 #include "bl_gemv_mma.cuh"
 #include "bl_gemv_stream.cuh"
+#include "bl_gemv_stream_mma.cuh"
 #include "bl_lnquant.cuh"
 #include "bl_pack.cuh"
 #include "bl_xnor.cuh"
@@ -46,7 +47,9 @@ struct DeviceState {
   // below num_sms / S (on B200: 74 / 33 / 15)
   int cluster_cap[9] = {};
   // clusters of 8 layer-stack decode CTAs that can be resident at once
+  // (single token; 8 and 16 token tiles)
   int stack_clusters = 0;
+  int stack_mma_clusters[2] = {0, 0};
 };
 DeviceState g_devices[kMaxDevices];
 
@@ -90,6 +93,8 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_lut_kernel<3>, 3 * kLutPageBytes) &&
               set_ts_smem<0>() && set_ts_smem<1>() && set_ts_smem<2>() &&
               set_smem(gemv_w1a16_stream_kernel, kStrSmemBytes) &&
+              set_smem(gemv_w1a16_stream_mma_kernel<8>, SmCfg<8>::kSmemBytes) &&
+              set_smem(gemv_w1a16_stream_mma_kernel<16>, SmCfg<16>::kSmemBytes) &&
               set_smem(gemm_ss_ste_kernel, kSsSmemBytes) &&
               set_smem(gemv_w1a16_mma_kernel<8, 16>, mma_smem_bytes(8, 16)) &&
               set_smem(gemv_w1a16_mma_kernel<16, 16>, mma_smem_bytes(16, 16)) &&
@@ -97,23 +102,29 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_mma_kernel<16, kMmaMaxSliceWords>, mma_smem_bytes(16, kMmaMaxSliceWords));
     if (!ok) cudaGetLastError();
     {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(kStrCluster, 1, 1);
-      cfg.blockDim = dim3(kStrThreads + 32, 1, 1);
-      cfg.dynamicSmemBytes = kStrSmemBytes;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = kStrCluster;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, gemv_w1a16_stream_kernel, &cfg) != cudaSuccess || n <= 0) {
-        cudaGetLastError();
-        n = 0;  // the stacked decode then reports BL_ERR_CUDA
-      }
-      st.stack_clusters = n;
+      // how many clusters of 8 of a stack kernel can be resident at once
+      auto stack_capacity = [](auto kernel, int smem) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kStrCluster, 1, 1);
+        cfg.blockDim = dim3(kStrThreads + 32, 1, 1);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kStrCluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+          cudaGetLastError();
+          n = 0;  // the stacked decode then reports BL_ERR_CUDA
+        }
+        return n;
+      };
+      st.stack_clusters = stack_capacity(gemv_w1a16_stream_kernel, kStrSmemBytes);
+      st.stack_mma_clusters[0] = stack_capacity(gemv_w1a16_stream_mma_kernel<8>, SmCfg<8>::kSmemBytes);
+      st.stack_mma_clusters[1] = stack_capacity(gemv_w1a16_stream_mma_kernel<16>, SmCfg<16>::kSmemBytes);
     }
     for (int S : {2, 4, 8}) {
       cudaLaunchConfig_t cfg = {};
@@ -140,13 +151,15 @@ int device_setup(int* num_sms) {
   return st.status;
 }
 
-int stack_cluster_capacity() {
+// resident clusters of the stack kernel for M tokens (1, <= 8, <= 16)
+int stack_cluster_capacity(int64_t M = 1) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return 0;
   }
-  return g_devices[dev].stack_clusters;
+  const DeviceState& st = g_devices[dev];
+  return M <= 1 ? st.stack_clusters : st.stack_mma_clusters[M <= 8 ? 0 : 1];
 }
 
 // co-resident cluster capacity of the current device for clusters of S GEMM CTAs
@@ -380,6 +393,29 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
   if (rc != BL_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
+  // short problems: LN, quantisation, products and rescale in one launch
+  if (!quant && !xq_in && M <= 16 && K <= kW1a8SmallMaxK && M * K <= kW1a8SmallMaxCodes &&
+      (!xq_out || aligned16(xq_out))) {
+    const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
+    const int m = int(M);
+    if (ternary) {
+      if (M <= 4)
+        bitlinear_small_kernel<4, true><<<grid, kGemvThreads, 0, s>>>(x, packed, beta, y, xq_out, gamma_out, acc_out, m, N, K);
+      else if (M <= 8)
+        bitlinear_small_kernel<8, true><<<grid, kGemvThreads, 0, s>>>(x, packed, beta, y, xq_out, gamma_out, acc_out, m, N, K);
+      else
+        bitlinear_small_kernel<16, true><<<grid, kGemvThreads, 0, s>>>(x, packed, beta, y, xq_out, gamma_out, acc_out, m, N, K);
+    } else {
+      if (M <= 4)
+        bitlinear_small_kernel<4, false><<<grid, kGemvThreads, 0, s>>>(x, packed, beta, y, xq_out, gamma_out, acc_out, m, N, K);
+      else if (M <= 8)
+        bitlinear_small_kernel<8, false><<<grid, kGemvThreads, 0, s>>>(x, packed, beta, y, xq_out, gamma_out, acc_out, m, N, K);
+      else
+        bitlinear_small_kernel<16, false><<<grid, kGemvThreads, 0, s>>>(x, packed, beta, y, xq_out, gamma_out, acc_out, m, N, K);
+    }
+    return launch_status();
+  }
+
   const int8_t* codes = xq_in;
   const double* gam = gamma_in;
   if (!xq_in) {
@@ -419,21 +455,30 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
     return BL_ERR_CUDA;
 
   if (M <= 16) {
-    const unsigned grid = static_cast<unsigned>(cdiv(N, kGemvRowsPerCta));
-    if (ternary) {
-      if (M <= 4)
-        gemv_w1a8_kernel<4, true><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
-      else if (M <= 8)
-        gemv_w1a8_kernel<8, true><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
-      else
-        gemv_w1a8_kernel<16, true><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
-    } else {
-      if (M <= 4)
-        gemv_w1a8_kernel<4, false><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
-      else if (M <= 8)
-        gemv_w1a8_kernel<8, false><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
-      else
-        gemv_w1a8_kernel<16, false><<<grid, kGemvThreads, 0, s>>>(codes, gam, packed, beta, y, acc_out, int(M), N, K);
+    // launched with programmatic serialisation: scheduled while the LN kernel
+    // runs, it waits for that kernel's codes before reading them
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cdiv(N, kGemvRowsPerCta)), 1, 1);
+    cfg.blockDim = dim3(kGemvThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int m = int(M);
+    cudaError_t e;
+    if (ternary)
+      e = M <= 4 ? cudaLaunchKernelEx(&cfg, gemv_w1a8_kernel<4, true>, codes, gam, packed, beta, y, acc_out, m, N, K)
+        : M <= 8 ? cudaLaunchKernelEx(&cfg, gemv_w1a8_kernel<8, true>, codes, gam, packed, beta, y, acc_out, m, N, K)
+                 : cudaLaunchKernelEx(&cfg, gemv_w1a8_kernel<16, true>, codes, gam, packed, beta, y, acc_out, m, N, K);
+    else
+      e = M <= 4 ? cudaLaunchKernelEx(&cfg, gemv_w1a8_kernel<4, false>, codes, gam, packed, beta, y, acc_out, m, N, K)
+        : M <= 8 ? cudaLaunchKernelEx(&cfg, gemv_w1a8_kernel<8, false>, codes, gam, packed, beta, y, acc_out, m, N, K)
+                 : cudaLaunchKernelEx(&cfg, gemv_w1a8_kernel<16, false>, codes, gam, packed, beta, y, acc_out, m, N, K);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
     }
     return launch_status();
   }
@@ -477,7 +522,7 @@ size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case BL_OP_W1A8_EX:
       return align256(size_t(M * K)) + align256(size_t(M) * sizeof(double)) +
              align256(size_t(M) * sizeof(LnTokenStats)) + 256;
-    case BL_OP_W1A16_STACK: return 256 + align256(size_t(N) * sizeof(uint32_t));
+    case BL_OP_W1A16_STACK: return 256 + align256(size_t(M > 1 ? M : 1) * size_t(N) * sizeof(uint32_t));
     case BL_OP_W1A16_BACKWARD: {
       const size_t Mp = size_t(cdiv(M, kSsUnit) * kSsUnit);
       return align256(size_t(M) * size_t(N) * 4) + align256(size_t(K) * size_t(N) / 4) +
@@ -601,7 +646,12 @@ int bitlinear_w1a8_ex(const uint16_t* x, const uint32_t* packed, const float* be
 
 int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const bl_stack_job* jobs,
                            int num_jobs, void* ws, size_t ws_bytes, void* stream) {
-  if (num_levels < 0 || num_jobs < 0) return BL_ERR_INVALID_ARG;
+  return bin_linear_w1a16_stack_batch(levels, num_levels, jobs, num_jobs, 1, ws, ws_bytes, stream);
+}
+
+int bin_linear_w1a16_stack_batch(const bl_stack_level* levels, int num_levels, const bl_stack_job* jobs,
+                                 int num_jobs, int64_t M, void* ws, size_t ws_bytes, void* stream) {
+  if (num_levels < 0 || num_jobs < 0 || M < 1 || M > 16) return BL_ERR_INVALID_ARG;
   if (num_levels == 0) return BL_OK;
   if (!levels || !jobs || !ws || !aligned16(ws)) return BL_ERR_INVALID_ARG;
   // level of every linear; the linears' outputs as byte ranges
@@ -624,18 +674,19 @@ int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const b
   }
   // every linear writes its own buffer
   std::sort(outs.begin(), outs.end());
+  const uintptr_t m2 = 2 * uintptr_t(M);  // bytes per element of a row, over the M tokens
   for (size_t t = 1; t < outs.size(); ++t)
-    if (outs[t].first < outs[t - 1].first + 2 * uintptr_t(jobs[outs[t - 1].second].N)) return BL_ERR_INVALID_ARG;
+    if (outs[t].first < outs[t - 1].first + m2 * uintptr_t(jobs[outs[t - 1].second].N)) return BL_ERR_INVALID_ARG;
   // the input of each level: a buffer written by no linear of the call, or
   // exactly the output of one linear of an earlier level
   std::vector<int> src(static_cast<size_t>(num_levels), -1);
   int64_t total_n = 0;
   for (int i = 0; i < num_levels; ++i) {
-    const uintptr_t x0 = reinterpret_cast<uintptr_t>(levels[i].x), x1 = x0 + 2 * uintptr_t(levels[i].K);
+    const uintptr_t x0 = reinterpret_cast<uintptr_t>(levels[i].x), x1 = x0 + m2 * uintptr_t(levels[i].K);
     auto it = std::upper_bound(outs.begin(), outs.end(), std::make_pair(x1, -1));
     if (it != outs.begin()) {
       const auto& o = *(it - 1);  // the last output starting before x ends
-      const uintptr_t o1 = o.first + 2 * uintptr_t(jobs[o.second].N);
+      const uintptr_t o1 = o.first + m2 * uintptr_t(jobs[o.second].N);
       if (o1 > x0) {  // overlaps
         if (o.first != x0 || jobs[o.second].N != levels[i].K || level_of[size_t(o.second)] >= i)
           return BL_ERR_INVALID_ARG;
@@ -644,11 +695,11 @@ int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const b
     }
   }
   for (int j = 0; j < num_jobs; ++j) total_n += level_of[size_t(j)] >= 0 ? jobs[j].N : 0;
-  if (ws_bytes < bl_workspace_bytes(BL_OP_W1A16_STACK, 0, total_n, 0)) return BL_ERR_INVALID_ARG;
+  if (ws_bytes < bl_workspace_bytes(BL_OP_W1A16_STACK, M, total_n, 0)) return BL_ERR_INVALID_ARG;
   int sms = 0;
   int rc = device_setup(&sms);
   if (rc != BL_OK) return rc;
-  const int G = stack_cluster_capacity();
+  const int G = stack_cluster_capacity(M);
   if (G < 1) return BL_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -674,7 +725,7 @@ int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const b
     const int j = src[size_t(i)];
     if (j >= 0 && launch_of[size_t(level_of[size_t(j)])] == launch_of[size_t(i)] && tag_off[size_t(j)] < 0) {
       tag_off[size_t(j)] = tagged_words;
-      tagged_words += jobs[j].N;
+      tagged_words += M * jobs[j].N;
     }
   }
   // ws: the abort word (first 256 bytes), then the tagged outputs; only
@@ -728,7 +779,7 @@ int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const b
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kStrCluster, static_cast<unsigned>(clusters), 1);
     cfg.blockDim = dim3(kStrThreads + 32, 1, 1);
-    cfg.dynamicSmemBytes = kStrSmemBytes;
+    cfg.dynamicSmemBytes = M == 1 ? kStrSmemBytes : (M <= 8 ? SmCfg<8>::kSmemBytes : SmCfg<16>::kSmemBytes);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -737,7 +788,11 @@ int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const b
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemv_w1a16_stream_kernel, P) != cudaSuccess) {
+    const int m = int(M);
+    const cudaError_t e = M == 1  ? cudaLaunchKernelEx(&cfg, gemv_w1a16_stream_kernel, P)
+                          : M <= 8 ? cudaLaunchKernelEx(&cfg, gemv_w1a16_stream_mma_kernel<8>, P, m)
+                                   : cudaLaunchKernelEx(&cfg, gemv_w1a16_stream_mma_kernel<16>, P, m);
+    if (e != cudaSuccess) {
       cudaGetLastError();
       return BL_ERR_CUDA;
     }

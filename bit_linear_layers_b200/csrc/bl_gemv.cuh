@@ -13,6 +13,7 @@
 #pragma once
 
 #include "bl_common.cuh"
+#include "bl_lnquant.cuh"
 
 namespace bl {
 
@@ -127,10 +128,10 @@ __device__ __forceinline__ uint32_t nibbles_to_ternary_i8(uint32_t plus, uint32_
 // kTernary: `packed` holds b1.58 weights, per 128-k block 4 words of the +1
 // plane then 4 of the -1 plane (row stride K/16 words)
 template <int MT, bool kTernary>
-__global__ void __launch_bounds__(kGemvThreads) gemv_w1a8_kernel(
-    const int8_t* __restrict__ xq, const double* __restrict__ gamma,
-    const uint32_t* __restrict__ packed, const float* __restrict__ beta, float* __restrict__ y,
-    int32_t* __restrict__ acc_out, int M, int64_t N, int64_t K) {
+__device__ __forceinline__ void w1a8_rows(const int8_t* __restrict__ xq, const double* __restrict__ gamma,
+                                          const uint32_t* __restrict__ packed, const float* __restrict__ beta,
+                                          float* __restrict__ y, int32_t* __restrict__ acc_out, int M, int64_t N,
+                                          int64_t K) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kGemvRowsPerCta + warp * kGemvRowsPerWarp;
   const int64_t words = K / 32;  // 32-k groups per row
@@ -184,6 +185,53 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_w1a8_kernel(
       }
     }
   }
+}
+
+
+// The dp4a GEMV as a kernel of its own, after the LN + quantisation kernel.
+// Launched with programmatic serialisation it is scheduled while that kernel
+// runs and waits for its results here.
+template <int MT, bool kTernary>
+__global__ void __launch_bounds__(kGemvThreads) gemv_w1a8_kernel(
+    const int8_t* __restrict__ xq, const double* __restrict__ gamma,
+    const uint32_t* __restrict__ packed, const float* __restrict__ beta, float* __restrict__ y,
+    int32_t* __restrict__ acc_out, int M, int64_t N, int64_t K) {
+  grid_dependency_wait();
+  w1a8_rows<MT, kTernary>(xq, gamma, packed, beta, y, acc_out, M, N, K);
+}
+
+// BitLinear for short problems in one launch ("BitNet b1.58" page, section
+// 1, Eq.(4)-(5), (7)-(8)): every CTA quantises all M tokens itself (one warp
+// per token, codes and gamma in shared memory), then runs the dp4a GEMV and
+// the rescale for its 32 rows. For M <= 16, K <= kW1a8SmallMaxK and M * K <=
+// kW1a8SmallMaxCodes, where repeating the LN in every CTA costs less than a
+// second launch. xq_out / gamma_out (written by CTA 0) and acc_out may be null.
+constexpr int kW1a8SmallMaxK = 1024;         // four 16-byte vectors per lane
+constexpr int kW1a8SmallMaxCodes = 16384;    // shared-memory codes
+template <int MT, bool kTernary>
+__global__ void __launch_bounds__(kGemvThreads) bitlinear_small_kernel(
+    const uint16_t* __restrict__ x, const uint32_t* __restrict__ packed, const float* __restrict__ beta,
+    float* __restrict__ y, int8_t* __restrict__ xq_out, double* __restrict__ gamma_out,
+    int32_t* __restrict__ acc_out, int M, int64_t N, int64_t K) {
+  __shared__ __align__(16) int8_t codes[kW1a8SmallMaxCodes];
+  __shared__ double gam[16];
+  const int warp = threadIdx.x >> 5;
+  for (int m = warp; m < M; m += kGemvWarps) {
+    if (K <= 256)
+      ln_quant_row_warp<1>(x + static_cast<int64_t>(m) * K, static_cast<int>(K), codes + m * K, &gam[m]);
+    else if (K <= 512)
+      ln_quant_row_warp<2>(x + static_cast<int64_t>(m) * K, static_cast<int>(K), codes + m * K, &gam[m]);
+    else
+      ln_quant_row_warp<4>(x + static_cast<int64_t>(m) * K, static_cast<int>(K), codes + m * K, &gam[m]);
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    if (xq_out)
+      for (int64_t i = threadIdx.x; i < M * K / 16; i += kGemvThreads)
+        reinterpret_cast<uint4*>(xq_out)[i] = reinterpret_cast<const uint4*>(codes)[i];
+    if (gamma_out && threadIdx.x < M) gamma_out[threadIdx.x] = gam[threadIdx.x];
+  }
+  w1a8_rows<MT, kTernary>(codes, gam, packed, beta, y, acc_out, M, N, K);
 }
 
 }  // namespace bl

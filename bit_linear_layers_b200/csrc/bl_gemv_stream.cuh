@@ -190,6 +190,54 @@ __device__ __forceinline__ bool str_next_slab(const StrJob* jobs, const StrLevel
   return true;
 }
 
+// The weight stream of one CTA (run by one thread): for every level, pass of
+// up to PASS slabs, table page and slab of the pass, in that order (the order
+// the compute warps consume them), one slot of tensor copies into the ring,
+// each slot reused once the compute warps have released it. Afterwards it
+// waits (bounded) for the last use of every slot, so that no copy is in
+// flight when the CTA exits.
+template <int PASS>
+__device__ __forceinline__ void str_produce(const StrParams& P, const StrLevel* lvs, const StrJob* jobs,
+                                            int num_levels, int cid, int G, uint32_t rank, uint8_t* ring,
+                                            uint64_t* full, uint64_t* empty) {
+  uint32_t issued = 0;
+  bool live = true;
+  for (int l = 0; l < num_levels; ++l) {
+    const StrLevel& lv = lvs[l];
+    StrRun run = str_run(jobs, lv, cid, G);
+    if (run.cur >= run.end) continue;
+    const LutWindow win = str_window(lv.K, rank);
+    const int np = str_pages(win);
+    while (true) {
+      StrSlab sl[PASS];
+      int npass = 0;
+      while (npass < PASS && str_next_slab(jobs, lv, run, sl[npass])) ++npass;
+      if (npass == 0) break;
+      for (int pg = 0; pg < np; ++pg) {
+        for (int i = 0; i < npass; ++i) {
+          const uint32_t slot = issued % kStrSlots;
+          if (issued >= static_cast<uint32_t>(kStrSlots) && live &&
+              !mbar_wait(smem_u32(&empty[slot]), ((issued / kStrSlots) - 1) & 1u, kWhereStackRing)) {
+            st_relaxed_gpu_u32(P.abort, 1u);
+            live = false;  // stop waiting; the outputs are undefined from here on
+          }
+          const uint32_t bar = smem_u32(&full[slot]);
+          const int boxes = (sl[i].nc() * kStrChunk + kStrBoxRows - 1) / kStrBoxRows;
+          mbar_arrive_expect_tx(bar, static_cast<uint32_t>(boxes) * kStrBoxRows * 16 * 4);
+          // x: window word (a multiple of 4 words = 16 bytes); y: row
+          for (int bx = 0; bx < boxes; ++bx)
+            tma_load_2d(smem_u32(ring + slot * kStrSlotBytes + bx * kStrBoxRows * 16 * 4), &P.maps[sl[i].j()], bar,
+                        win.a0 + 16 * pg, sl[i].row0 + bx * kStrBoxRows);
+          ++issued;
+        }
+      }
+    }
+  }
+  const uint32_t first = issued > static_cast<uint32_t>(kStrSlots) ? issued - kStrSlots : 0u;
+  for (uint32_t k = first; k < issued; ++k)
+    if (!mbar_wait(smem_u32(&full[k % kStrSlots]), (k / kStrSlots) & 1u, kWhereStackRing)) break;
+}
+
 // Warps 0..15 compute (kStrThreads threads); warp 16 streams the weights.
 // (17 warps: one SM sub-partition hosts 5 of them, which caps registers at 96.)
 __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_kernel(const __grid_constant__ StrParams P) {
@@ -235,45 +283,7 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_kernel(
 
   if (warp == kWarps) {
     // ---- the weight stream (one thread): slots in processing order ----
-    if (lane == 0) {
-      uint32_t issued = 0;
-      bool live = true;
-      for (int l = 0; l < num_levels; ++l) {
-        const StrLevel& lv = lvs[l];
-        StrRun run = str_run(jobs, lv, cid, G);
-        if (run.cur >= run.end) continue;
-        const LutWindow win = str_window(lv.K, rank);
-        const int np = str_pages(win);
-        while (true) {
-          StrSlab sl[kStrPass];
-          int npass = 0;
-          while (npass < kStrPass && str_next_slab(jobs, lv, run, sl[npass])) ++npass;
-          if (npass == 0) break;
-          for (int pg = 0; pg < np; ++pg) {
-            for (int i = 0; i < npass; ++i) {
-              const uint32_t slot = issued % kStrSlots;
-              if (issued >= static_cast<uint32_t>(kStrSlots) && live &&
-                  !mbar_wait(smem_u32(&empty[slot]), ((issued / kStrSlots) - 1) & 1u, kWhereStackRing)) {
-                st_relaxed_gpu_u32(P.abort, 1u);
-                live = false;  // stop waiting; the outputs are undefined from here on
-              }
-              const uint32_t bar = smem_u32(&full[slot]);
-              const int boxes = (sl[i].nc() * kStrChunk + kStrBoxRows - 1) / kStrBoxRows;
-              mbar_arrive_expect_tx(bar, static_cast<uint32_t>(boxes) * kStrBoxRows * 16 * 4);
-              // x: window word (a multiple of 4 words = 16 bytes); y: row
-              for (int bx = 0; bx < boxes; ++bx)
-                tma_load_2d(smem_u32(ring + slot * kStrSlotBytes + bx * kStrBoxRows * 16 * 4), &P.maps[sl[i].j()], bar,
-                            win.a0 + 16 * pg, sl[i].row0 + bx * kStrBoxRows);
-              ++issued;
-            }
-          }
-        }
-      }
-      // no copy may be in flight at exit: wait (bounded) for the last use of each slot
-      const uint32_t first = issued > static_cast<uint32_t>(kStrSlots) ? issued - kStrSlots : 0u;
-      for (uint32_t k = first; k < issued; ++k)
-        if (!mbar_wait(smem_u32(&full[k % kStrSlots]), (k / kStrSlots) & 1u, kWhereStackRing)) break;
-    }
+    if (lane == 0) str_produce<kStrPass>(P, lvs, jobs, num_levels, cid, G, rank, ring, full, empty);
     __syncwarp();
   } else {
     uint32_t q = 0;  // slots consumed

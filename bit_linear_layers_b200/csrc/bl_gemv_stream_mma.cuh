@@ -1,0 +1,259 @@
+// Decode of a batch of 2..16 tokens through a stack of binarized linear
+// layers in one persistent launch ("FBI-LLM" page, FBI-linear paragraph:
+// y_mj = bf16(alpha_j * sum_k sign(W_jk) x_mk) for every linear, the levels
+// one after another).
+//
+// The same machinery as the single-token stack kernel (bl_gemv_stream.cuh):
+// clusters of 8 CTAs splitting K into slices, balanced runs of 16-row chunks
+// cut into slabs, a producer warp streaming 16 KB weight slots into a ring by
+// tensor copies, outputs published as tagged words, an 8-way exchange of the
+// slice partials through the row owners' inboxes. What differs is the
+// arithmetic: with up to 16 tokens the products run on the warp-level
+// m16n8k16 bf16 MMA, as in the few-token GEMV (bl_gemv_mma.cuh): a warp's 16
+// rows (g and g + 8 of the A fragment) over the CTA's K slice, the signs
+// turned into +-1 bf16 A registers in place (r = b | b << 15, shift, mask,
+// xor), the tokens the 8-wide N side (one or two MMAs per 16 k), fp32
+// accumulation. No lookup table is built, so each level needs only its input
+// slice in shared memory ([token][k - 32 s0], padded so that a B fragment's
+// 32 lanes hit 32 banks), one slab per pass.
+//
+// Tagged buffers hold [token][N] words; the exchange carries 16 tokens per
+// row. Waits are bounded as in the single-token kernel.
+#pragma once
+
+#include "bl_gemv_mma.cuh"
+#include "bl_gemv_stream.cuh"
+
+namespace bl {
+
+constexpr int kSmMaxSlice = 48;                                  // words of a slice (K <= 12288)
+__host__ __device__ constexpr int sm_x_pitch(int mt) { (void)mt; return kSmMaxSlice * 64 + 16; }  // bytes per token
+template <int MT>
+struct SmCfg {
+  static constexpr int kInbox = 2 * kStrCluster * 32 * MT;        // floats: [pass % 2][src rank][owned row][token]
+  static constexpr int kXBytes = MT * sm_x_pitch(MT);
+  static constexpr int kSmemBytes = kStrSlots * kStrSlotBytes + kXBytes + kInbox * 4;  // dynamic
+};
+
+template <int MT>
+__global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_mma_kernel(const __grid_constant__ StrParams P,
+                                                                                     int M) {
+  using C = SmCfg<MT>;
+  constexpr int H = MT / 8;  // n-halves of the token tile
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* ring = smem;                                          // kStrSlots x 16 KB
+  uint8_t* xs = smem + kStrSlots * kStrSlotBytes;                // [token][slice k] bf16, padded rows
+  float* inbox = reinterpret_cast<float*>(xs + C::kXBytes);
+  __shared__ __align__(8) uint64_t inbox_full[2];
+  __shared__ __align__(8) uint64_t full[kStrSlots];
+  __shared__ __align__(8) uint64_t empty[kStrSlots];
+  __shared__ StrLevel lvs[kStrMaxLevels];
+  __shared__ StrJob jobs[kStrMaxJobs];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t rank = cluster_ctarank();
+  const int G = static_cast<int>(gridDim.y), cid = static_cast<int>(blockIdx.y);
+  constexpr int kOwned = kStrRows / kStrCluster;  // 32 rows of a slab per owner
+  constexpr int kWarps = kStrThreads / 32;
+  const int pitch = sm_x_pitch(MT);
+
+  for (int i = tid; i < P.num_levels * static_cast<int>(sizeof(StrLevel) / 16); i += blockDim.x)
+    reinterpret_cast<uint4*>(lvs)[i] = reinterpret_cast<const uint4*>(P.lv)[i];
+  for (int i = tid; i < P.num_jobs * static_cast<int>(sizeof(StrJob) / 16); i += blockDim.x)
+    reinterpret_cast<uint4*>(jobs)[i] = reinterpret_cast<const uint4*>(P.jobs)[i];
+  // tokens past M stay zero in the input slices for the whole launch
+  for (int i = tid; i < C::kXBytes / 16; i += blockDim.x) reinterpret_cast<uint4*>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (tid == 0) {
+    mbar_init(smem_u32(&inbox_full[0]), 1);
+    mbar_init(smem_u32(&inbox_full[1]), 1);
+    for (int s = 0; s < kStrSlots; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), kWarps);
+    }
+    fence_mbar_init();
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  const int num_levels = P.num_levels;
+
+  if (warp == kWarps) {
+    if (lane == 0) str_produce<1>(P, lvs, jobs, num_levels, cid, G, rank, ring, full, empty);
+    __syncwarp();
+  } else {
+    uint32_t q = 0, n = 0;
+    bool ok = true;
+    for (int l = 0; l < num_levels; ++l) {
+      const StrLevel& lv = lvs[l];
+      StrRun run = str_run(jobs, lv, cid, G);
+      if (run.cur >= run.end) continue;
+      const LutWindow win = str_window(lv.K, rank);
+      const int np = str_pages(win);
+
+      // ---- the slice of every token's input: xs[m][k - 32 s0] ----
+      {
+        const int e0 = win.s0 * 32, ne = win.sw * 32;
+        if (lv.xt) {
+          // the loads of up to kBatch vectors per thread are all in flight
+          // before any is checked, so a level's input costs about one L2
+          // round trip (plus a re-poll of what was not yet published)
+          constexpr int kBatch = 6;
+          const int per_tok = ne / 4, total = M * per_tok;
+          for (int v0 = tid; v0 < total; v0 += kBatch * kStrThreads) {
+            uint4 tv[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+              const int v = v0 + b * kStrThreads;
+              if (v < total) {
+                const int m = v / per_tok, e = (v - m * per_tok) * 4;
+                tv[b] = ld_relaxed_gpu_v4(lv.xt + static_cast<int64_t>(m) * lv.K + e0 + e);
+              }
+            }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+              const int v = v0 + b * kStrThreads;
+              if (v >= total) continue;
+              const int m = v / per_tok, e = (v - m * per_tok) * 4;
+              if (!((tv[b].x & tv[b].y & tv[b].z & tv[b].w) & kStrReady) && ok) {
+                const uint32_t* src = lv.xt + static_cast<int64_t>(m) * lv.K + e0 + e;
+                const uint64_t t0 = global_timer_ns();
+                do {
+                  tv[b] = ld_relaxed_gpu_v4(src);
+                  if ((tv[b].x & tv[b].y & tv[b].z & tv[b].w) & kStrReady) break;
+                  if (ld_relaxed_gpu_u32(P.abort) != 0u) {
+                    ok = false;
+                    break;
+                  }
+                  if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+                    record_error(BL_ERR_TIMEOUT, kWhereStackLevel);
+                    st_relaxed_gpu_u32(P.abort, 1u);
+                    ok = false;
+                    break;
+                  }
+                } while (true);
+              }
+              uint2 v2;
+              v2.x = (tv[b].x & 0xFFFFu) | (tv[b].y << 16);
+              v2.y = (tv[b].z & 0xFFFFu) | (tv[b].w << 16);
+              *reinterpret_cast<uint2*>(xs + m * pitch + 2 * e) = v2;
+            }
+          }
+        } else {
+          const int per_tok = ne / 8;
+          for (int v = tid; v < M * per_tok; v += kStrThreads) {
+            const int m = v / per_tok, e = (v - m * per_tok) * 8;
+            *reinterpret_cast<uint4*>(xs + m * pitch + 2 * e) =
+                *reinterpret_cast<const uint4*>(lv.x + static_cast<int64_t>(m) * lv.K + e0 + e);
+          }
+        }
+      }
+      consumers_sync();
+
+      StrSlab sl;
+      while (str_next_slab(jobs, lv, run, sl)) {
+        // bytes of partials this CTA receives: 8 ranks x MT tokens x 4 bytes per owned live row
+        if (tid == 0) {
+          const int r = sl.nc() * kStrChunk - static_cast<int>(rank) * kOwned;
+          const uint32_t rows = r <= 0 ? 0u : (r >= kOwned ? static_cast<uint32_t>(kOwned) : static_cast<uint32_t>(r));
+          mbar_arrive_expect_tx(smem_u32(&inbox_full[n & 1u]), rows * kStrCluster * MT * 4);
+        }
+        // owners: thread (token m = tid / 32, row r = tid % 32) of the slab
+        const int om = tid / kOwned, orr = tid % kOwned;
+        const int orow_s = static_cast<int>(rank) * kOwned + orr;  // row within the slab
+        const StrJob& jb = jobs[sl.j()];
+        const bool owner = om < M && orow_s < sl.nc() * kStrChunk && sl.row0 + orow_s < jb.N;
+        const int orow = sl.row0 + orow_s;
+        const float oalpha = owner ? jb.alpha[orow] : 0.f;
+
+        float acc[H][4];
+#pragma unroll
+        for (int hh = 0; hh < H; ++hh)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[hh][i] = 0.f;
+        const uint32_t sh_lo = 15 - 2 * t, sh_hi = 7 - 2 * t;
+        for (int pg = 0; pg < np; ++pg) {
+          const uint32_t slot = q % kStrSlots;
+          if (ok && !mbar_wait(smem_u32(&full[slot]), (q / kStrSlots) & 1u, kWhereStackRing)) {
+            st_relaxed_gpu_u32(P.abort, 1u);
+            ok = false;
+          }
+          if (warp < sl.nc()) {
+            const uint32_t* sw = reinterpret_cast<const uint32_t*>(ring + slot * kStrSlotBytes);
+            const int ra = warp * kStrChunk + g;  // rows ra and ra + 8 of the slab
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+              const int wi = pg * 16 + w;
+              if (wi < win.lo() || wi >= win.hi()) continue;  // uniform across the warp
+              const uint32_t wa = sw[ra * 16 + w], wb = sw[(ra + 8) * 16 + w];
+              const int kb = (wi - win.lo()) * 64;  // byte offset of the word's 32 inputs in a token row
+#pragma unroll
+              for (int o = 0; o < 2; ++o) {
+                const uint32_t ba = (wa >> (16 * o)) & 0xFFFFu, bb = (wb >> (16 * o)) & 0xFFFFu;
+                const uint32_t rra = ba | (ba << 15), rrb = bb | (bb << 15);
+                const uint32_t a[4] = {((rra << sh_lo) & 0x80008000u) ^ 0xBF80BF80u,
+                                       ((rrb << sh_lo) & 0x80008000u) ^ 0xBF80BF80u,
+                                       ((rra << sh_hi) & 0x80008000u) ^ 0xBF80BF80u,
+                                       ((rrb << sh_hi) & 0x80008000u) ^ 0xBF80BF80u};
+#pragma unroll
+                for (int hh = 0; hh < H; ++hh) {
+                  const uint8_t* p = xs + (8 * hh + g) * pitch + kb + o * 32 + 4 * t;
+                  mma_bf16_16816(acc[hh], a, *reinterpret_cast<const uint32_t*>(p),
+                                 *reinterpret_cast<const uint32_t*>(p + 16));
+                }
+              }
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
+          ++q;
+        }
+
+        // ---- partials to the rows' owners: rows ra, ra + 8 of warp w belong to rank w / 2 ----
+        if (warp < sl.nc()) {
+          const uint32_t owner_rank = static_cast<uint32_t>(warp >> 1);
+          const uint32_t bar = map_to_rank(smem_u32(&inbox_full[n & 1u]), owner_rank);
+          const int r0 = (warp * kStrChunk + g) & (kOwned - 1);
+          float* ib = inbox + (n & 1u) * (C::kInbox / 2);
+#pragma unroll
+          for (int hh = 0; hh < H; ++hh) {
+            const int tok = 8 * hh + 2 * t;
+            const uint32_t sa = smem_u32(&ib[(static_cast<int>(rank) * kOwned + r0) * MT + tok]);
+            const uint32_t sb = smem_u32(&ib[(static_cast<int>(rank) * kOwned + r0 + 8) * MT + tok]);
+            st_async_v2_f32(map_to_rank(sa, owner_rank), acc[hh][0], acc[hh][1], bar);
+            st_async_v2_f32(map_to_rank(sb, owner_rank), acc[hh][2], acc[hh][3], bar);
+          }
+        }
+        uint16_t yv = 0;
+        bool got = false;
+        if (tid < MT * kOwned) {
+          if (ok) {
+            got = mbar_wait(smem_u32(&inbox_full[n & 1u]), (n >> 1) & 1u, kWhereStackInbox);
+            if (!got) {
+              st_relaxed_gpu_u32(P.abort, 1u);
+              ok = false;
+            }
+          }
+          if (got && owner) {
+            const float* in = inbox + (n & 1u) * (C::kInbox / 2) + orr * MT + om;
+            float sum = 0.f;
+#pragma unroll
+            for (int r = 0; r < kStrCluster; ++r) sum += in[r * kOwned * MT];
+            yv = float_to_bf16_bits(oalpha * sum);
+          }
+        }
+        if (got && owner) {
+          const int64_t o = static_cast<int64_t>(om) * jb.N + orow;
+          if (jb.tagged) st_relaxed_gpu_u32(jb.tagged + o, kStrReady | yv);  // publish first
+          jb.y[o] = yv;
+        }
+        // the owners have read this pass's inbox before any warp pushes the next pass
+        consumers_sync();
+        ++n;
+      }
+    }
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+}
+
+}  // namespace bl

@@ -98,6 +98,9 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_kernel(const uint16_t* __
   __shared__ float shm[2][kLnWarps];
   const int64_t m = blockIdx.x;
   if (m >= M) return;  // uniform per CTA
+  // a kernel launched after this one with programmatic serialisation (the
+  // few-token GEMV) may be scheduled now; it waits for this grid's results
+  grid_dependents_launch();
   const uint4* row = reinterpret_cast<const uint4*>(x + m * K);
   const int64_t nvec = K / 8;  // 8 bf16 per 16-byte load
 
@@ -326,6 +329,88 @@ __global__ void __launch_bounds__(kLnThreads) ln_quant_tensor_kernel(const uint1
       }
     }
     out[i] = make_uint2(codes[0], codes[1]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The same LN + per-token absmax quantisation of one token by one warp, for
+// short rows (K <= 256 * NVW): the statistics are reduced by warp shuffles
+// (a different summation order from ln_quant_kernel: gamma may differ in its
+// last bits, within the same bound), the code decision is quant_code with the
+// same fp64 fallback. `codes` may point to shared memory.
+template <int NVW>
+__device__ __forceinline__ void ln_quant_row_warp(const uint16_t* __restrict__ xrow, int K, int8_t* codes,
+                                                  double* gamma_out) {
+  const int lane = threadIdx.x & 31;
+  const uint4* row = reinterpret_cast<const uint4*>(xrow);
+  const int nvec = K / 8;
+  uint4 cache[NVW];
+#pragma unroll
+  for (int u = 0; u < NVW; ++u) {
+    const int i = lane + 32 * u;
+    cache[u] = i < nvec ? row[i] : make_uint4(0u, 0u, 0u, 0u);
+  }
+  double s0 = 0.0, s1 = 0.0;
+  float xmax = -INFINITY, xmin = INFINITY;
+#pragma unroll
+  for (int u = 0; u < NVW; ++u) {
+    if (lane + 32 * u < nvec) {
+      const uint32_t h[4] = {cache[u].x, cache[u].y, cache[u].z, cache[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s0 += bf16_to_double(h[j] & 0xFFFFu);
+        s1 += bf16_to_double(h[j] >> 16);
+        const float a = bf16_lo(h[j]), b = bf16_hi(h[j]);
+        xmax = fmaxf(xmax, fmaxf(a, b));
+        xmin = fminf(xmin, fminf(a, b));
+      }
+    }
+  }
+  xmax = warp_max(xmax);
+  xmin = -warp_max(-xmin);
+  const double mu = warp_sum(s0 + s1) / static_cast<double>(K);
+  double q0 = 0.0, q1 = 0.0;
+#pragma unroll
+  for (int u = 0; u < NVW; ++u) {
+    if (lane + 32 * u < nvec) {
+      const uint32_t h[4] = {cache[u].x, cache[u].y, cache[u].z, cache[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const double d0 = bf16_to_double(h[j] & 0xFFFFu) - mu;
+        const double d1 = bf16_to_double(h[j] >> 16) - mu;
+        q0 = fma(d0, d0, q0);
+        q1 = fma(d1, d1, q1);
+      }
+    }
+  }
+  const double sq = warp_sum(q0 + q1);
+  const double dmax = fmax(static_cast<double>(xmax) - mu, mu - static_cast<double>(xmin));
+  LnQuantParams p;
+  p.mu = mu;
+  p.root = sqrt(sq / static_cast<double>(K) + kLnEps);
+  p.gamma = dmax / p.root;
+  p.mu_hi = static_cast<float>(mu);
+  p.mu_lo = static_cast<float>(mu - static_cast<double>(p.mu_hi));
+  p.c32 = dmax > 0.0 ? static_cast<float>(128.0 / dmax) : 0.f;
+  if (lane == 0) *gamma_out = p.gamma;
+  uint2* out = reinterpret_cast<uint2*>(codes);
+#pragma unroll
+  for (int u = 0; u < NVW; ++u) {
+    const int i = lane + 32 * u;
+    if (i < nvec) {
+      const uint32_t h[4] = {cache[u].x, cache[u].y, cache[u].z, cache[u].w};
+      uint32_t packed_codes[2] = {0u, 0u};
+      if (dmax > 0.0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int q0c = quant_code(bf16_lo(h[j]), p);
+          const int q1c = quant_code(bf16_hi(h[j]), p);
+          const uint32_t pair = (static_cast<uint32_t>(q0c) & 0xFFu) | ((static_cast<uint32_t>(q1c) & 0xFFu) << 8);
+          packed_codes[j >> 1] |= pair << (16 * (j & 1));
+        }
+      }
+      out[i] = make_uint2(packed_codes[0], packed_codes[1]);
+    }
   }
 }
 

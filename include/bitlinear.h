@@ -67,7 +67,7 @@ extern "C" {
 #define BL_OP_PACK_TERNARY 4
 #define BL_OP_W158A8 5
 #define BL_OP_W1A8_EX 6 /* bitlinear_w1a8_ex with a per-tensor quantiser */
-#define BL_OP_W1A16_STACK 7 /* bin_linear_w1a16_stack (N = total outputs; M, K ignored) */
+#define BL_OP_W1A16_STACK 7 /* bin_linear_w1a16_stack(_batch) (M tokens, N = total outputs; K ignored) */
 #define BL_OP_W1A16_BACKWARD 8 /* bin_linear_w1a16_backward */
 
 /* Library ABI version (this header: 1). */
@@ -200,6 +200,19 @@ typedef struct bl_stack_level {
 } bl_stack_level;
 int bin_linear_w1a16_stack(const bl_stack_level* levels, int num_levels, const bl_stack_job* jobs,
                            int num_jobs, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bin_linear_w1a16_stack_batch -- bin_linear_w1a16_stack for a decode batch
+ * of M tokens (1 <= M <= 16): every level's x is [M x K] and every linear's y
+ * [M x N] (bf16, row-major), y[m][j] = bf16(alpha[j] * sum_k s_jk x[m][k])
+ * for each token. The rules on inputs and outputs are those of
+ * bin_linear_w1a16_stack, with buffers of M rows. M == 1 is exactly
+ * bin_linear_w1a16_stack; for M >= 2 the products run on the warp-level
+ * tensor-core MMA (fp32 accumulation), with the same weight streaming. ws:
+ * bl_workspace_bytes(BL_OP_W1A16_STACK, M, total_N, 0) bytes.
+ */
+int bin_linear_w1a16_stack_batch(const bl_stack_level* levels, int num_levels, const bl_stack_job* jobs,
+                                 int num_jobs, int64_t M, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * bitlinear_w1a8 -- BitNet BitLinear forward ("BitNet b1.58" page,

@@ -7,6 +7,9 @@ layers in one persistent launch) on the GPU.
   level, and inputs produced by earlier levels;
 * bit-identical to bin_linear_w1a16 called layer by layer where that call
   also splits K eight ways (K = 4096 and 11008, the 7B shapes);
+* decode batches of 2..16 tokens (bin_linear_w1a16_stack_batch): every token
+  of every level against the oracle, and bit-identical to the per-layer
+  few-token MMA GEMV at the 7B shapes;
 * stacks longer than one launch (more than 96 levels or 144 linears);
 * the argument checks."""
 import ctypes
@@ -35,32 +38,35 @@ def _linear(oracle, N, K, seed):
 
 
 def _check_level(oracle, x_dev, linears, what):
-    """linears: (packed_np, alpha_np, y_dev) of one level; x_dev the level input."""
+    """linears: (packed_np, alpha_np, y_dev) of one level; x_dev the level input ([K] or [M, K])."""
     import synthetic
-    xb = synthetic.bf16_bits(x_dev.reshape(1, -1))
-    K = xb.shape[1]
+    K = x_dev.shape[-1]
+    xb = synthetic.bf16_bits(x_dev.reshape(-1, K))
+    M = xb.shape[0]
     for i, (packed, alpha, y) in enumerate(linears):
-        y_ref = oracle.w1a16(xb, packed, alpha, K).ravel()
+        y_ref = oracle.w1a16(xb, packed, alpha, K)
         N = packed.shape[0]
-        check_w1a16(bf16_to_f64(y.reshape(1, -1)).ravel(), y_ref, alpha, xb, np.zeros(N, np.int64), np.arange(N),
-                    what=f"{what} linear {i}")
+        ms, js = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
+        check_w1a16(bf16_to_f64(y.reshape(M, N))[ms, js].ravel(), y_ref[ms, js].ravel(), alpha, xb,
+                    ms.ravel(), js.ravel(), what=f"{what} linear {i}")
 
 
-def _run_and_check(bl, oracle, spec, seed0):
+def _run_and_check(bl, oracle, spec, seed0, M=1):
     """spec: list of levels, each (K, [N...], src) where src is None (a fresh
-    input) or (level, linear) whose output feeds this level."""
+    input) or (level, linear) whose output feeds this level; M tokens."""
     import synthetic
     levels, host, outs = [], [], []
     for li, (K, Ns, src) in enumerate(spec):
         if src is None:
-            x = synthetic.activations(1, K, seed0 + 1000 * li).reshape(K).cuda()
+            x = synthetic.activations(M, K, seed0 + 1000 * li).cuda()
+            x = x.reshape(K) if M == 1 else x
         else:
             x = outs[src[0]][src[1]]
-            assert x.numel() == K
+            assert x.numel() == M * K
         lins, hl, ys = [], [], []
         for j, N in enumerate(Ns):
             dp, da, packed, alpha = _linear(oracle, N, K, seed0 + 1000 * li + 7 * j + 1)
-            y = torch.full((N,), float("nan"), dtype=torch.bfloat16, device="cuda")
+            y = torch.full((N,) if M == 1 else (M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
             lins.append((dp, da, y))
             hl.append((packed, alpha, y))
             ys.append(y)
@@ -112,6 +118,47 @@ def test_stack_matches_layer_by_layer_at_7b_shapes(bl, oracle):
         cur = bl.bin_linear_w1a16(cur, dp, da)
         ref.append(cur.reshape(N))
     torch.cuda.synchronize()
+    for i, (a, b) in enumerate(zip(ys, ref)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"level {i} differs"
+
+
+@pytest.mark.parametrize("M", [2, 5, 8, 9, 16])
+def test_stack_batch_chained_levels(bl, oracle, M):
+    # the miniature block stack of test_stack_chained_levels, M tokens at once
+    spec = []
+    for layer in range(2):
+        base = len(spec)
+        src = None if layer == 0 else (base - 1, 0)
+        spec.append((1024, [1024, 1024, 1024], src))
+        spec.append((1024, [1024], (base, 2)))
+        spec.append((1024, [2816, 2816], (base + 1, 0)))
+        spec.append((2816, [1024], (base + 2, 1)))
+    _run_and_check(bl, oracle, spec, seed0=31 + M, M=M)
+
+
+def test_stack_batch_each_page_count(bl, oracle):
+    # slices of 1..48 words, ragged N, 16 tokens
+    spec = [(256, [100], None), (4096, [300, 1], None), (11008, [700], None), (12288, [257], None)]
+    _run_and_check(bl, oracle, spec, seed0=41, M=16)
+
+
+@pytest.mark.parametrize("M", [8, 16])
+def test_stack_batch_matches_layer_by_layer_at_7b_shapes(bl, oracle, M):
+    """The few-token MMA GEMV splits K eight ways too: identical bits."""
+    import synthetic
+    shapes = [(4096, 4096), (4096, 4096), (4096, 11008), (11008, 4096)]  # (K, N)
+    x0 = synthetic.activations(M, 4096, 6).cuda()
+    mats = [_linear(oracle, N, K, 60 + i)[:2] for i, (K, N) in enumerate(shapes)]
+    ys = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _, N in shapes]
+    levels = [(x0, [(mats[0][0], mats[0][1], ys[0])]), (ys[0], [(mats[1][0], mats[1][1], ys[1])]),
+              (ys[1], [(mats[2][0], mats[2][1], ys[2])]), (ys[2], [(mats[3][0], mats[3][1], ys[3])])]
+    bl.W1A16Stack(levels).run()
+    ref, cur = [], x0
+    for (dp, da), (K, N) in zip(mats, shapes):
+        cur = bl.bin_linear_w1a16(cur, dp, da)
+        ref.append(cur)
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
     for i, (a, b) in enumerate(zip(ys, ref)):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"level {i} differs"
 
