@@ -14,8 +14,9 @@
 // turned into +-1 bf16 A registers in place (r = b | b << 15, shift, mask,
 // xor), the tokens the 8-wide N side (one or two MMAs per 16 k), fp32
 // accumulation. No lookup table is built, so each level needs only its input
-// slice in shared memory ([token][k - 32 s0], padded so that a B fragment's
-// 32 lanes hit 32 banks), one slab per pass.
+// slice in shared memory ([token][k - 32 s0], each 32-k word permuted so that
+// an A register is one shift and one LOP3 of a packed word and a B fragment
+// one 64-bit load; rows padded so those loads hit 32 banks), one slab per pass.
 //
 // Tagged buffers hold [token][N] words; the exchange carries 16 tokens per
 // row. Waits are bounded as in the single-token kernel.
@@ -27,7 +28,22 @@
 namespace bl {
 
 constexpr int kSmMaxSlice = 48;                                  // words of a slice (K <= 12288)
-__host__ __device__ constexpr int sm_x_pitch(int mt) { (void)mt; return kSmMaxSlice * 64 + 16; }  // bytes per token
+// bytes per token row of the staged inputs: the slice plus 32 bytes, so that
+// the 64-bit B-fragment loads of a half-warp (4 tokens x 4 lanes) hit 32 banks
+__host__ __device__ constexpr int sm_x_pitch(int mt) { (void)mt; return kSmMaxSlice * 64 + 32; }
+
+// Order of the inputs within a 32-k word as staged for the MMAs. The dot
+// product does not depend on the order of k, so the inputs are permuted (and
+// the signs read at the matching bits) to make the A registers cheap: lane t's
+// register j of 16-k chunk o takes the signs of bits b and b + 16 of the
+// packed word, b = 4t + 2o + j, which one shift brings to the two bf16 sign
+// positions (15 and 31). Staged position p (0..31) of a word holds input
+//   k(p) = b + 16 (p & 1),  b = 4 ((p >> 2) & 3) + 2 (p >> 4) + ((p >> 1) & 1),
+// so that lane t's B fragment of chunk o (the MMA's k = 2t, 2t + 1, 2t + 8,
+// 2t + 9) is the 4 consecutive positions 16 o + 4 t .. + 3.
+__host__ __device__ constexpr int sm_perm_k(int p) {
+  return 4 * ((p >> 2) & 3) + 2 * (p >> 4) + ((p >> 1) & 1) + 16 * (p & 1);
+}
 template <int MT>
 struct SmCfg {
   static constexpr int kInbox = 2 * kStrCluster * 32 * MT;        // floats: [pass % 2][src rank][owned row][token]
@@ -90,36 +106,25 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_mma_ker
       const LutWindow win = str_window(lv.K, rank);
       const int np = str_pages(win);
 
-      // ---- the slice of every token's input: xs[m][k - 32 s0] ----
+      // ---- the slice of every token's input, each 32-k word in the
+      // permuted order above: xs[m][32 w + p] = x[m][32 (s0 + w) + k(p)] ----
       {
-        const int e0 = win.s0 * 32, ne = win.sw * 32;
-        if (lv.xt) {
-          // the loads of up to kBatch vectors per thread are all in flight
-          // before any is checked, so a level's input costs about one L2
-          // round trip (plus a re-poll of what was not yet published)
-          constexpr int kBatch = 6;
-          const int per_tok = ne / 4, total = M * per_tok;
-          for (int v0 = tid; v0 < total; v0 += kBatch * kStrThreads) {
-            uint4 tv[kBatch];
+        const int e0 = win.s0 * 32, blocks = M * win.sw;  // (token, word) blocks
+        for (int blk = tid; blk < blocks; blk += kStrThreads) {
+          const int m = blk / win.sw, w = blk - m * win.sw;
+          uint32_t v[16];  // bf16 pairs of inputs k = 2i, 2i + 1
+          if (lv.xt) {
+            const uint32_t* src = lv.xt + static_cast<int64_t>(m) * lv.K + e0 + 32 * w;
+            uint4 tv[8];
 #pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-              const int v = v0 + b * kStrThreads;
-              if (v < total) {
-                const int m = v / per_tok, e = (v - m * per_tok) * 4;
-                tv[b] = ld_relaxed_gpu_v4(lv.xt + static_cast<int64_t>(m) * lv.K + e0 + e);
-              }
-            }
+            for (int i = 0; i < 8; ++i) tv[i] = ld_relaxed_gpu_v4(src + 4 * i);
 #pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-              const int v = v0 + b * kStrThreads;
-              if (v >= total) continue;
-              const int m = v / per_tok, e = (v - m * per_tok) * 4;
-              if (!((tv[b].x & tv[b].y & tv[b].z & tv[b].w) & kStrReady) && ok) {
-                const uint32_t* src = lv.xt + static_cast<int64_t>(m) * lv.K + e0 + e;
+            for (int i = 0; i < 8; ++i) {
+              if (!((tv[i].x & tv[i].y & tv[i].z & tv[i].w) & kStrReady) && ok) {
                 const uint64_t t0 = global_timer_ns();
                 do {
-                  tv[b] = ld_relaxed_gpu_v4(src);
-                  if ((tv[b].x & tv[b].y & tv[b].z & tv[b].w) & kStrReady) break;
+                  tv[i] = ld_relaxed_gpu_v4(src + 4 * i);
+                  if ((tv[i].x & tv[i].y & tv[i].z & tv[i].w) & kStrReady) break;
                   if (ld_relaxed_gpu_u32(P.abort) != 0u) {
                     ok = false;
                     break;
@@ -132,19 +137,30 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_mma_ker
                   }
                 } while (true);
               }
-              uint2 v2;
-              v2.x = (tv[b].x & 0xFFFFu) | (tv[b].y << 16);
-              v2.y = (tv[b].z & 0xFFFFu) | (tv[b].w << 16);
-              *reinterpret_cast<uint2*>(xs + m * pitch + 2 * e) = v2;
+              v[2 * i] = (tv[i].x & 0xFFFFu) | (tv[i].y << 16);
+              v[2 * i + 1] = (tv[i].z & 0xFFFFu) | (tv[i].w << 16);
+            }
+          } else {
+            const uint4* src = reinterpret_cast<const uint4*>(lv.x + static_cast<int64_t>(m) * lv.K + e0 + 32 * w);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 q4 = src[i];
+              v[4 * i] = q4.x, v[4 * i + 1] = q4.y, v[4 * i + 2] = q4.z, v[4 * i + 3] = q4.w;
             }
           }
-        } else {
-          const int per_tok = ne / 8;
-          for (int v = tid; v < M * per_tok; v += kStrThreads) {
-            const int m = v / per_tok, e = (v - m * per_tok) * 8;
-            *reinterpret_cast<uint4*>(xs + m * pitch + 2 * e) =
-                *reinterpret_cast<const uint4*>(lv.x + static_cast<int64_t>(m) * lv.K + e0 + e);
+          // output pair (p, p + 1), p even: inputs k(p) and k(p) + 16
+          uint32_t o[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k0 = sm_perm_k(2 * i);  // even input index? take its half of the pair
+            const uint32_t lo = (k0 & 1) ? (v[k0 >> 1] >> 16) : (v[k0 >> 1] & 0xFFFFu);
+            const int k1 = k0 + 16;
+            const uint32_t hi = (k1 & 1) ? (v[k1 >> 1] & 0xFFFF0000u) : (v[k1 >> 1] << 16);
+            o[i] = lo | hi;
           }
+          uint4* dst = reinterpret_cast<uint4*>(xs + m * pitch + 64 * w);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
       }
       consumers_sync();
@@ -157,8 +173,9 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_mma_ker
           const uint32_t rows = r <= 0 ? 0u : (r >= kOwned ? static_cast<uint32_t>(kOwned) : static_cast<uint32_t>(r));
           mbar_arrive_expect_tx(smem_u32(&inbox_full[n & 1u]), rows * kStrCluster * MT * 4);
         }
-        // owners: thread (token m = tid / 32, row r = tid % 32) of the slab
-        const int om = tid / kOwned, orr = tid % kOwned;
+        // owners: thread (row r = tid / MT, token m = tid % MT) of the slab
+        // (tokens fastest: a warp's inbox reads are consecutive words)
+        const int om = tid % MT, orr = tid / MT;
         const int orow_s = static_cast<int>(rank) * kOwned + orr;  // row within the slab
         const StrJob& jb = jobs[sl.j()];
         const bool owner = om < M && orow_s < sl.nc() * kStrChunk && sl.row0 + orow_s < jb.N;
@@ -170,7 +187,8 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_mma_ker
         for (int hh = 0; hh < H; ++hh)
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[hh][i] = 0.f;
-        const uint32_t sh_lo = 15 - 2 * t, sh_hi = 7 - 2 * t;
+        // lane t's A register j of chunk o: signs of bits 4t + 2o + j and + 16
+        const uint32_t sh00 = 15 - 4 * t, sh01 = 14 - 4 * t, sh10 = 13 - 4 * t, sh11 = 12 - 4 * t;
         for (int pg = 0; pg < np; ++pg) {
           const uint32_t slot = q % kStrSlots;
           if (ok && !mbar_wait(smem_u32(&full[slot]), (q / kStrSlots) & 1u, kWhereStackRing)) {
@@ -180,25 +198,40 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_mma_ker
           if (warp < sl.nc()) {
             const uint32_t* sw = reinterpret_cast<const uint32_t*>(ring + slot * kStrSlotBytes);
             const int ra = warp * kStrChunk + g;  // rows ra and ra + 8 of the slab
+            // one 16-bit half (o) of window word w (bits wa of row ra, wb of
+            // row ra + 8): 16 k, H MMAs
+            auto chunk = [&](uint32_t wa, uint32_t wb, int w, int o) {
+              const uint32_t s0 = o ? sh10 : sh00, s1 = o ? sh11 : sh01;
+              // bit b -> bit 15 and bit b + 16 -> bit 31; set bit -> +1 (0x3F80)
+              const uint32_t a[4] = {((wa << s0) & 0x80008000u) ^ 0xBF80BF80u, ((wb << s0) & 0x80008000u) ^ 0xBF80BF80u,
+                                     ((wa << s1) & 0x80008000u) ^ 0xBF80BF80u, ((wb << s1) & 0x80008000u) ^ 0xBF80BF80u};
+              const int kb = (pg * 16 + w - win.lo()) * 64 + o * 32 + 8 * t;  // lane's 4 staged inputs
 #pragma unroll
-            for (int w = 0; w < 16; ++w) {
-              const int wi = pg * 16 + w;
-              if (wi < win.lo() || wi >= win.hi()) continue;  // uniform across the warp
-              const uint32_t wa = sw[ra * 16 + w], wb = sw[(ra + 8) * 16 + w];
-              const int kb = (wi - win.lo()) * 64;  // byte offset of the word's 32 inputs in a token row
+              for (int hh = 0; hh < H; ++hh) {
+                const uint2 bv = *reinterpret_cast<const uint2*>(xs + (8 * hh + g) * pitch + kb);
+                mma_bf16_16816(acc[hh], a, bv.x, bv.y);
+              }
+            };
+            const bool full_page = pg * 16 >= win.lo() && pg * 16 + 16 <= win.hi();
+            // the page's words of both rows, four at a time
 #pragma unroll
-              for (int o = 0; o < 2; ++o) {
-                const uint32_t ba = (wa >> (16 * o)) & 0xFFFFu, bb = (wb >> (16 * o)) & 0xFFFFu;
-                const uint32_t rra = ba | (ba << 15), rrb = bb | (bb << 15);
-                const uint32_t a[4] = {((rra << sh_lo) & 0x80008000u) ^ 0xBF80BF80u,
-                                       ((rrb << sh_lo) & 0x80008000u) ^ 0xBF80BF80u,
-                                       ((rra << sh_hi) & 0x80008000u) ^ 0xBF80BF80u,
-                                       ((rrb << sh_hi) & 0x80008000u) ^ 0xBF80BF80u};
+            for (int c = 0; c < 4; ++c) {
+              const uint4 va = *reinterpret_cast<const uint4*>(sw + ra * 16 + 4 * c);
+              const uint4 vb = *reinterpret_cast<const uint4*>(sw + (ra + 8) * 16 + 4 * c);
+              const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+              if (full_page) {  // every word live: straight-line code
 #pragma unroll
-                for (int hh = 0; hh < H; ++hh) {
-                  const uint8_t* p = xs + (8 * hh + g) * pitch + kb + o * 32 + 4 * t;
-                  mma_bf16_16816(acc[hh], a, *reinterpret_cast<const uint32_t*>(p),
-                                 *reinterpret_cast<const uint32_t*>(p + 16));
+                for (int i = 0; i < 4; ++i) {
+                  chunk(wa[i], wb[i], 4 * c + i, 0);
+                  chunk(wa[i], wb[i], 4 * c + i, 1);
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int wi = pg * 16 + 4 * c + i;
+                  if (wi < win.lo() || wi >= win.hi()) continue;  // uniform across the warp
+                  chunk(wa[i], wb[i], 4 * c + i, 0);
+                  chunk(wa[i], wb[i], 4 * c + i, 1);
                 }
               }
             }

@@ -8,8 +8,7 @@ layers in one persistent launch) on the GPU.
 * bit-identical to bin_linear_w1a16 called layer by layer where that call
   also splits K eight ways (K = 4096 and 11008, the 7B shapes);
 * decode batches of 2..16 tokens (bin_linear_w1a16_stack_batch): every token
-  of every level against the oracle, and bit-identical to the per-layer
-  few-token MMA GEMV at the 7B shapes;
+  of every level against the oracle, at small and 7B shapes;
 * stacks longer than one launch (more than 96 levels or 144 linears);
 * the argument checks."""
 import ctypes
@@ -143,24 +142,11 @@ def test_stack_batch_each_page_count(bl, oracle):
 
 
 @pytest.mark.parametrize("M", [8, 16])
-def test_stack_batch_matches_layer_by_layer_at_7b_shapes(bl, oracle, M):
-    """The few-token MMA GEMV splits K eight ways too: identical bits."""
-    import synthetic
-    shapes = [(4096, 4096), (4096, 4096), (4096, 11008), (11008, 4096)]  # (K, N)
-    x0 = synthetic.activations(M, 4096, 6).cuda()
-    mats = [_linear(oracle, N, K, 60 + i)[:2] for i, (K, N) in enumerate(shapes)]
-    ys = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _, N in shapes]
-    levels = [(x0, [(mats[0][0], mats[0][1], ys[0])]), (ys[0], [(mats[1][0], mats[1][1], ys[1])]),
-              (ys[1], [(mats[2][0], mats[2][1], ys[2])]), (ys[2], [(mats[3][0], mats[3][1], ys[3])])]
-    bl.W1A16Stack(levels).run()
-    ref, cur = [], x0
-    for (dp, da), (K, N) in zip(mats, shapes):
-        cur = bl.bin_linear_w1a16(cur, dp, da)
-        ref.append(cur)
-    torch.cuda.synchronize()
-    assert bl.device_error() == (0, 0)
-    for i, (a, b) in enumerate(zip(ys, ref)):
-        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"level {i} differs"
+def test_stack_batch_at_7b_shapes(bl, oracle, M):
+    """A 7B block's four levels (K = 4096 and 11008, the slices of 16 and 43
+    words) at 8 and 16 tokens, every output against the oracle."""
+    spec = [(4096, [4096, 512], None), (4096, [4096], (0, 0)), (4096, [11008], (1, 0)), (11008, [4096], (2, 0))]
+    _run_and_check(bl, oracle, spec, seed0=60 + M, M=M)
 
 
 def test_stack_longer_than_one_launch(bl, oracle):
