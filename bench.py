@@ -2,7 +2,8 @@
 """Benchmark of the binarized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|w1a8|w158a8|w1a1] [--no-secondary]
+                    [--workload decode|prefill|backward|w1a8|w1a8_single|w158a8|w1a8_tensor|w1a1]
+                    [--no-secondary] [--probe-int8]
 
 Workloads (a step is one pass of the layer over one batch of synthetic input):
 
@@ -16,13 +17,19 @@ Workloads (a step is one pass of the layer over one batch of synthetic input):
   rescale) on the 1.3B shapes, 512 tokens, 2048->5632 then 5632->2048, in
   TOP/s against the int8 tensor peak;
 * ``w158a8``: the same with BitNet b1.58 ternary weights;
+* ``w1a8_tensor``: the same with the per-tensor Eq.(5) quantiser;
 * ``w1a1``: XNOR/popcount products of packed +-1 operands at the same shapes,
-  against a population-count (integer ALU) roofline.
+  against a population-count (integer ALU) roofline;
+* ``w1a8_single``: one small BitLinear layer, M=4 tokens, K=N=256 (one fused
+  launch), in tokens per second;
+* ``backward``: the straight-through FBI-linear backward (dx, dW, dalpha) of
+  the 7B MLP up-projection at 2048 tokens, in TFLOP/s.
 
 Each workload keeps R distinct copies of its weights and activations whose
 total is more than twice the 126 MB L2, and step i uses copy i % R, so no step
 finds its inputs in L2. After W untimed warm-up steps, K steps are captured
-in one CUDA graph and timed with CUDA events on the launching stream; with N
+in one CUDA graph and timed with CUDA events recorded as the graph's first and
+last nodes on the launching stream; with N
 ranks (torchrun) every rank runs its own replica (no data-path collective)
 and the time is the max over ranks.
 
@@ -811,29 +818,32 @@ WORKLOADS = {w.name: w for w in (Decode, Prefill, Backward, W1A8, W1A8Single, W1
 
 
 def _capture(step, first, count, stream):
+    """A CUDA graph of `count` steps whose first and last nodes record two
+    timing events (external event nodes), so that the events bracket exactly
+    the steps' device work and not the graph's own launch."""
     import torch
     graph = torch.cuda.CUDAGraph()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
     with torch.cuda.stream(stream):
         with torch.cuda.graph(graph, stream=stream):
+            e0.record(stream)
             for i in range(count):
                 step(first + i)
+            e1.record(stream)
     torch.cuda.synchronize()
     graph.replay()  # untimed replay: the graph's first launch uploads it
     torch.cuda.synchronize()
-    return graph
+    return graph, (e0, e1)
 
 
-def _timed_replay(graph, dev, world):
+def _timed_replay(captured, dev, world):
     import torch
+    graph, (e0, e1) = captured
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    launch_stream = torch.cuda.current_stream(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(launch_stream)
     graph.replay()
-    e1.record(launch_stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -1278,7 +1288,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = WORKLOADS[args.workload]()
     config = dict(wl.config)
-    config["timing"] = "K steps in one CUDA graph, CUDA events on the launching stream"
+    config["timing"] = ("K steps in one CUDA graph, timed by CUDA events recorded as the graph's first and last "
+                        "nodes (the launching stream)")
     config["parallelism"] = f"replicas x{world}"
 
     if args.impl == "reference":

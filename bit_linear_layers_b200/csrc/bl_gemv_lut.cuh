@@ -245,6 +245,11 @@ __global__ void __launch_bounds__(kLutThreads, NP == 1 ? 2 : 1) gemv_w1a16_lut_k
   // the owners' scales (not written by the previous kernel either)
   const int orow = row0 + static_cast<int>(rank) * rows_per_cta + static_cast<int>(threadIdx.x);
   const float oalpha = (threadIdx.x < rows_per_cta && orow < N) ? alpha[orow] : 0.f;
+  // ask L2 for this slice of x now: a prefetch reads nothing into the CTA
+  // and L2 is coherent, so it is safe even while the previous kernel is still
+  // writing x; the loads after the wait then find it there
+  if (threadIdx.x < (win.sw * 64 + 127) / 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(x + static_cast<int64_t>(win.s0) * 32 + threadIdx.x * 64) : "memory");
 
   // x may be produced by the previous kernel on the stream
   grid_dependency_wait();
