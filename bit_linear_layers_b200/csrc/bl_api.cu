@@ -526,7 +526,8 @@ size_t bl_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) {
     case BL_OP_W1A16_BACKWARD: {
       const size_t Mp = size_t(cdiv(M, kSsUnit) * kSsUnit);
       return align256(size_t(M) * size_t(N) * 4) + align256(size_t(K) * size_t(N) / 4) +
-             align256(size_t(K) * 4) + align256(size_t(K) * Mp * 2) + align256(size_t(N) * Mp * 2);
+             align256(size_t(K) * 4) + align256(size_t(K) * Mp * 2) + align256(size_t(N) * Mp * 2) +
+             align256(size_t(K / kSsRowsA) * size_t(N) * 4);
     }
     default: return 0;
   }
@@ -837,6 +838,8 @@ int bin_linear_w1a16_backward(const uint16_t* x, const uint32_t* packed, const f
   auto* xt = reinterpret_cast<uint16_t*>(w);
   w += align256(size_t(K) * size_t(Mp) * 2);
   auto* dyt = reinterpret_cast<uint16_t*>(w);
+  w += align256(size_t(N) * size_t(Mp) * 2);
+  auto* part = reinterpret_cast<float*>(w);  // [K / 128][N] signed partial sums for dalpha
   const unsigned ew_grid = static_cast<unsigned>(sms * 8);
   if (dx) {
     // dx = [hi | lo] x [S^T | S^T] through the forward path (unit scales)
@@ -866,10 +869,12 @@ int bin_linear_w1a16_backward(const uint16_t* x, const uint32_t* packed, const f
       return BL_ERR_CUDA;
     const int64_t tiles = (K / kSsRowsA) * cdiv(N, kSsRowsB);
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-    gemm_ss_ste_kernel<<<grid, kSsThreads, kSsSmemBytes, s>>>(tm_a, tm_b, int(K), int(N), int(Mp), dw);
+    // dW = alpha P and the per-tile signed sums for dalpha come out of the GEMM's epilogue
+    gemm_ss_ste_kernel<<<grid, kSsThreads, kSsSmemBytes, s>>>(tm_a, tm_b, int(K), int(N), int(Mp), alpha, packed,
+                                                               dw, part);
     if ((rc = launch_status()) != BL_OK) return rc;
-    const int64_t fblocks = cdiv(N, 8) < int64_t(sms) * 16 ? cdiv(N, 8) : int64_t(sms) * 16;
-    ste_finalize_kernel<<<static_cast<unsigned>(fblocks), 256, 0, s>>>(dw, packed, alpha, N, K, dalpha);
+    const int64_t dblocks = cdiv(N, 256) < int64_t(sms) * 4 ? cdiv(N, 256) : int64_t(sms) * 4;
+    ste_dalpha_kernel<<<static_cast<unsigned>(dblocks), 256, 0, s>>>(part, K / kSsRowsA, N, dalpha);
     if ((rc = launch_status()) != BL_OK) return rc;
   }
   return BL_OK;

@@ -15,7 +15,9 @@
 // transpose_pack_dup_kernel writes S^T (each row twice) in the packed layout.
 // P is a plain tcgen05 GEMM with both operands in shared memory (TMA,
 // 128-byte swizzle), computed as D[k][j] = sum_m X^T[k][m] dY^T[j][m] so that
-// each warp's stores of a column j are contiguous in P's row j.
+// each warp's stores of a column j are contiguous in P's row j. P itself is
+// never stored: its epilogue writes dW = alpha_j P and, per 128-k tile, the
+// signed sums sum_k s_jk P_jk, which a small kernel adds up into dalpha.
 #pragma once
 
 #include "bl_common.cuh"
@@ -91,27 +93,15 @@ __global__ void fill_f32_kernel(float* __restrict__ p, int64_t n, float v) {
     p[i] = v;
 }
 
-// In place over P [N][K] (fp32): dW_jk = alpha_j P_jk, and dalpha_j =
-// sum_k s_jk P_jk (fp64 sum in a fixed order). One warp per row.
-__global__ void ste_finalize_kernel(float* __restrict__ pw, const uint32_t* __restrict__ packed,
-                                    const float* __restrict__ alpha, int64_t N, int64_t K,
-                                    float* __restrict__ dalpha) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t kw_count = K / 32;
-  for (int64_t j = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; j < N; j += warps) {
-    const float a = alpha[j];
-    float* row = pw + j * K;
-    const uint32_t* bits = packed + j * kw_count;
+// dalpha_j = sum over the 128-k tiles of the partials the dW GEMM wrote
+// (part[t][j] = sum over tile t of s_jk P_jk), added in tile order in fp64.
+__global__ void ste_dalpha_kernel(const float* __restrict__ part, int64_t tiles, int64_t N,
+                                  float* __restrict__ dalpha) {
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < N;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     double s = 0.0;
-    for (int64_t kw = 0; kw < kw_count; ++kw) {
-      const uint32_t w = bits[kw];
-      const float p = row[kw * 32 + lane];
-      s += ((w >> lane) & 1u) ? static_cast<double>(p) : -static_cast<double>(p);
-      row[kw * 32 + lane] = a * p;
-    }
-    s = warp_sum(s);
-    if (lane == 0) dalpha[j] = static_cast<float>(s);
+    for (int64_t t = 0; t < tiles; ++t) s += static_cast<double>(part[t * N + j]);
+    dalpha[j] = static_cast<float>(s);
   }
 }
 
@@ -128,17 +118,27 @@ constexpr int kSsStageBytes = kSsABytes + kSsBBytes;  // 48 KB
 constexpr int kSsSmemBytes = kSsStages * kSsStageBytes + 1024;
 
 // tm_a: X^T [Kdim][Mp] bf16, box 64 x 128; tm_b: dY^T [Ndim][Mp] bf16, box 64 x 256.
-// Writes P[j][k] (fp32, row pitch Kdim) for j < Ndim. Two accumulators in
-// tensor memory, so the epilogue of one tile overlaps the next tile's MMAs.
+// P[j][k] = sum_m dY[m][j] X[m][k]. Writes dW[j][k] = alpha_j P[j][k] (fp32,
+// row pitch Kdim) for j < Ndim, and for every 128-k tile t the signed sums
+// part[t][j] = sum_{k in t} s_jk P[j][k] (fp32; `packed` holds s, [Ndim][Kdim/32]),
+// which ste_dalpha_kernel adds up. Two accumulators in tensor memory, so the
+// epilogue of one tile overlaps the next tile's MMAs.
 __global__ void __launch_bounds__(kSsThreads, 1) gemm_ss_ste_kernel(const __grid_constant__ CUtensorMap tm_a,
                                                                     const __grid_constant__ CUtensorMap tm_b,
                                                                     int Kdim, int Ndim, int Mp,
-                                                                    float* __restrict__ P) {
+                                                                    const float* __restrict__ alpha,
+                                                                    const uint32_t* __restrict__ packed,
+                                                                    float* __restrict__ P, float* __restrict__ part) {
   extern __shared__ uint8_t ss_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ss_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   __shared__ __align__(8) uint64_t full[kSsStages], empty[kSsStages], d_full[2], d_empty[2];
   __shared__ uint32_t tmem_base_sh;
+  // the epilogue's view of a tile: scales, sign words [j][k word] and the
+  // four warps' signed partial sums
+  __shared__ float alpha_sh[kSsRowsB];
+  __shared__ uint32_t bits_sh[kSsRowsB][kSsRowsA / 32];
+  __shared__ float part_sh[4][kSsRowsB];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_a = Kdim / kSsRowsA;
   const int tiles_b = (Ndim + kSsRowsB - 1) / kSsRowsB;
@@ -217,13 +217,30 @@ __global__ void __launch_bounds__(kSsThreads, 1) gemm_ss_ste_kernel(const __grid
       }
     }
   } else if (warp >= 4) {
-    const int q = warp & 3;
+    const int q = warp & 3, et = threadIdx.x - 128;  // epilogue thread 0..127
+    const int kwords = Kdim / 32;
+    auto epi_sync = [] { asm volatile("bar.sync 2, 128;" ::: "memory"); };
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
       const uint32_t ab = tcount & 1u;
       const int k0 = (tile % tiles_a) * kSsRowsA, j0 = (tile / tiles_a) * kSsRowsB;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&d_full[ab]), (tcount / 2) & 1, kWhereSsEpilogue));
-      if (!ok) break;
+      // this tile's scales and sign words (rows past Ndim: 0)
+      for (int i = et; i < kSsRowsB; i += 128) alpha_sh[i] = j0 + i < Ndim ? alpha[j0 + i] : 0.f;
+      for (int i = et; i < kSsRowsB * (kSsRowsA / 32); i += 128) {
+        const int jj = i / (kSsRowsA / 32), w = i % (kSsRowsA / 32);
+        bits_sh[jj][w] = j0 + jj < Ndim ? packed[static_cast<int64_t>(j0 + jj) * kwords + k0 / 32 + w] : 0u;
+      }
+      // (the barrier also publishes the staging) the four warps leave together
+      // if a wait gave up
+      const bool waited = mbar_wait(smem_u32(&d_full[ab]), (tcount / 2) & 1, kWhereSsEpilogue);
+      uint32_t all_ok;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+          "bar.red.and.pred q, 2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(all_ok)
+          : "r"(static_cast<uint32_t>(waited))
+          : "memory");
+      if (!all_ok) break;
       tc_fence_after_sync();
       const int k = k0 + q * 32 + lane;  // this thread's row of D = column of P
 #pragma unroll 1
@@ -234,6 +251,13 @@ __global__ void __launch_bounds__(kSsThreads, 1) gemm_ss_ste_kernel(const __grid
         tmem_wait_ld();
         const int jc = j0 + cc * 32;
         float* pp = P + static_cast<int64_t>(jc) * Kdim + k;
+        float sg[32];  // s_jk P_jk of this lane's k for the chunk's 32 rows j
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float pv = __uint_as_float(r[i]);
+          sg[i] = ((bits_sh[cc * 32 + i][q] >> lane) & 1u) ? pv : -pv;
+          r[i] = __float_as_uint(alpha_sh[cc * 32 + i] * pv);
+        }
         if (jc + 32 <= Ndim) {
 #pragma unroll
           for (int i = 0; i < 32; ++i, pp += Kdim) *pp = __uint_as_float(r[i]);
@@ -242,10 +266,28 @@ __global__ void __launch_bounds__(kSsThreads, 1) gemm_ss_ste_kernel(const __grid
           for (int i = 0; i < 32; ++i, pp += Kdim)
             if (jc + i < Ndim) *pp = __uint_as_float(r[i]);
         }
+        // reduce-scatter over the warp's 32 k: lane L ends with row jc + L
+#pragma unroll
+        for (int d = 16, n = 32; d >= 1; d >>= 1, n >>= 1) {
+          const bool upper = (lane & d) != 0;
+#pragma unroll
+          for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? sg[i] : sg[i + n / 2];
+            const float keep = upper ? sg[i + n / 2] : sg[i];
+            sg[i] = keep + __shfl_xor_sync(0xffffffffu, send, d);
+          }
+        }
+        part_sh[q][cc * 32 + lane] = sg[0];
       }
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&d_empty[ab]));
+      epi_sync();  // the four warps' partials are in part_sh; the tile's staging is free again
+      for (int i = et; i < kSsRowsB; i += 128)
+        if (j0 + i < Ndim)
+          part[static_cast<int64_t>(k0 / kSsRowsA) * Ndim + j0 + i] =
+              (part_sh[0][i] + part_sh[1][i]) + (part_sh[2][i] + part_sh[3][i]);
+      epi_sync();  // part_sh has been read before the next tile writes it
     }
   }
 
