@@ -2,7 +2,8 @@
 """Benchmark of the binarized linear layers on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|backward|w1a8|w1a8_single|w158a8|w1a8_tensor|w1a1]
+                    [--workload decode|prefill|backward|w1a8|w1a8_single|w158a8|w1a8_tensor|w1a1|
+                                decode_stack|decode_stack16]
                     [--no-secondary] [--probe-int8]
 
 Workloads (a step is one pass of the layer over one batch of synthetic input):
@@ -23,11 +24,15 @@ Workloads (a step is one pass of the layer over one batch of synthetic input):
 * ``w1a8_single``: one small BitLinear layer, M=4 tokens, K=N=256 (one fused
   launch), in tokens per second;
 * ``backward``: the straight-through FBI-linear backward (dx, dW, dalpha) of
-  the 7B MLP up-projection at 2048 tokens, in TFLOP/s.
+  the 7B MLP up-projection at 2048 tokens, in TFLOP/s;
+* ``decode_stack`` / ``decode_stack16``: one token step of a 7B-shaped
+  FBI-LLM's 224 linears (32 layers, each layer's outputs feeding the next) at
+  batch 1 / 16 as one stacked call, in tokens per second, against HBM.
 
 Each workload keeps R distinct copies of its weights and activations whose
 total is more than twice the 126 MB L2, and step i uses copy i % R, so no step
-finds its inputs in L2. After W untimed warm-up steps, K steps are captured
+finds its inputs in L2 (the stacked decode streams 0.8 GB of signs per step:
+one copy). After W untimed warm-up steps, K steps are captured
 in one CUDA graph and timed with CUDA events recorded as the graph's first and
 last nodes on the launching stream; with N
 ranks (torchrun) every rank runs its own replica (no data-path collective)
@@ -549,6 +554,7 @@ class W1A8Single(Workload):
     dtype = "s8"
     kernel = "bitlinear_small_kernel<4,false> (one fused launch per call)"
     sources = [CSRC + "bl_gemv.cuh", CSRC + "bl_lnquant.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = "bitlinear_small_w1a8_single_4x256x256.traffic.json"
     roof_unit = "GB/s"
     rotate = 18000  # 14 KB per copy: 250 MB, about twice the L2
 
@@ -811,7 +817,138 @@ class W1A1(Workload):
             self.o.w1a1(a, b, K)
 
 
-WORKLOADS = {w.name: w for w in (Decode, Prefill, Backward, W1A8, W1A8Single, W158A8, W1A8Tensor, W1A1)}
+
+_LLAMA7B = {}
+
+
+def llama7b_layers(dev):
+    """The packed signs and scales of all 224 linears of a 7B-shaped model
+    (32 layers x q, k, v, o, gate, up, down), built once per process."""
+    if dev not in _LLAMA7B:
+        import bit_linear_layers_b200 as bl
+        import synthetic
+        layers = []
+        for layer in range(synthetic.LLAMA7B_LAYERS):
+            mats = []
+            for idx, (K, N) in enumerate(synthetic.LLAMA7B_LAYER):
+                W = synthetic.weights(N, K, seed=5000 + 16 * layer + idx, device=dev)
+                mats.append(bl.bin_pack(W, bl.BL_PACK_FBI))
+                del W
+            layers.append(mats)
+        _LLAMA7B[dev] = layers
+    return _LLAMA7B[dev]
+
+
+class DecodeStack(Workload):
+    """Decode of a 7B-shaped FBI-LLM's linears (32 layers x q, k, v, o,
+    gate, up, down; 0.8 GB of packed signs, more than L2) at batch B, one
+    bin_linear_w1a16_stack(_batch) call per token step: 128 levels per
+    step (q, k, v from the layer input; o from v; gate, up from o; down
+    from up, which feeds the next layer), every linear writing a buffer of
+    its own. A step is one token step of all B tokens through all 224
+    linears."""
+    name = "decode_stack"
+    B = 1
+    metric = ("7B-shaped FBI-LLM linear-only decode tok/s at batch 1 (W1A16, 32 layers x 7 linears, "
+              "one stacked call per token step)")
+    unit, scale, bound = "tok/s", 1.0, "hbm"
+    roof_unit = "GB/s"
+    kernel = "gemv_w1a16_stream_kernel (15 clusters of 8 CTAs, persistent; 96 + 32 levels per step)"
+    sources = [CSRC + "bl_gemv_stream.cuh", CSRC + "bl_gemv_lut.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = "gemv_w1a16_stream_7b_decode_batch1.traffic.json"
+    launches_per_step = 2
+
+    def __init__(self):
+        import synthetic
+        B = self.B
+        self.linears = [(K, N) for _ in range(synthetic.LLAMA7B_LAYERS) for K, N in synthetic.LLAMA7B_LAYER]
+        self.packed_b = sum(N * K // 8 for K, N in self.linears)
+        self.alg_b = sum(N * K // 8 + 4 * N + 2 * B * K + 2 * B * N for K, N in self.linears)
+        self.config = {"workload": f"all 224 linears of a 7B-shaped FBI-LLM (32 layers x q,k,v,o 4096x4096; gate,up "
+                                   f"4096->11008; down 11008->4096), W1A16 decode at batch {B}",
+                       "batch": B, "layers": synthetic.LLAMA7B_LAYERS, "levels_per_step": 4 * synthetic.LLAMA7B_LAYERS,
+                       "packed_bytes_per_step": self.packed_b, "algorithmic_bytes_per_step": self.alg_b,
+                       "l2": f"inputs larger than L2: {self.packed_b / 1e6:.0f} MB of packed signs streamed per step",
+                       "call": "bin_linear_w1a16_stack" + ("" if B == 1 else "_batch") +
+                               " (a zero-fill of the tagged outputs, then the persistent kernel per 96 levels)"}
+
+    def units_per_step(self):
+        return float(self.B)  # tokens
+
+    def achieved(self, per_step_s):
+        return self.alg_b / per_step_s / 1e9  # all bytes the step must move
+
+    def peak(self, peaks, timed_s):
+        return peaks["hbm_gbs"], "hbm_gbs"
+
+    def setup(self, dev, rank):
+        import torch
+        import bit_linear_layers_b200 as bl
+        import synthetic
+        B = self.B
+        layers = llama7b_layers(dev)
+        shp = (lambda n: (n,)) if B == 1 else (lambda n: (B, n))
+        self.x = synthetic.activations(B, 4096, seed=77 + 7 * rank, device=dev).reshape(shp(4096))
+        levels, cur = [], self.x
+        for mats in layers:
+            q, k, v, o, h = (torch.empty(shp(4096), dtype=torch.bfloat16, device=dev) for _ in range(5))
+            g, u = (torch.empty(shp(11008), dtype=torch.bfloat16, device=dev) for _ in range(2))
+            levels.append((cur, [(mats[0][0], mats[0][1], q), (mats[1][0], mats[1][1], k),
+                                 (mats[2][0], mats[2][1], v)]))
+            levels.append((v, [(mats[3][0], mats[3][1], o)]))
+            levels.append((o, [(mats[4][0], mats[4][1], g), (mats[5][0], mats[5][1], u)]))
+            levels.append((u, [(mats[6][0], mats[6][1], h)]))
+            cur = h
+        self.h = cur
+        self.stack = bl.W1A16Stack(levels)
+        self.xh = [self.x.cpu().pin_memory() for _ in range(2)]
+        self.hh = [torch.empty_like(self.h, device="cpu").pin_memory() for _ in range(2)]
+        self.h2d, self.d2h = 2 * B * 4096, 2 * B * 4096
+
+    def step(self, i):
+        self.stack.run()
+
+    def e2e_step(self, i):
+        self.x.copy_(self.xh[i % 2], non_blocking=True)
+        self.stack.run()
+        self.hh[i % 2].copy_(self.h, non_blocking=True)
+
+    # oracle: output rows [0, 256) of each linear of layer 0, all B tokens, per call
+    ORACLE_ROWS = 256
+
+    def oracle_setup(self):
+        import oracle as oracle_pkg
+        import synthetic
+        self.o = oracle_pkg.get()
+        self.olin, work = [], 0.0
+        for idx, (K, N) in enumerate(synthetic.LLAMA7B_LAYER):
+            W = synthetic.weights(self.ORACLE_ROWS, K, seed=5000 + idx).numpy()
+            packed, alpha = self.o.pack_fbi(W)
+            x = synthetic.bf16_bits(synthetic.activations(self.B, K, seed=77 + idx))
+            self.olin.append((x, packed, alpha, K))
+            work += self.ORACLE_ROWS * K
+        self.oracle_sample = (f"output rows 0..{self.ORACLE_ROWS - 1} of each of the 7 linear shapes of a layer for "
+                              f"{self.B} token(s) per call (single-threaded C oracle, fp64)")
+        return self.B * work / sum(N * K for K, N in self.linears)  # token steps per call
+
+    def oracle_call(self):
+        for x, packed, alpha, K in self.olin:
+            self.o.w1a16(x, packed, alpha, K)
+
+
+class DecodeStack16(DecodeStack):
+    name = "decode_stack16"
+    B = 16
+    metric = ("7B-shaped FBI-LLM linear-only decode tok/s at batch 16 (W1A16, 32 layers x 7 linears, "
+              "one stacked call per token step)")
+    kernel = "gemv_w1a16_stream_mma_kernel<16> (15 clusters of 8 CTAs, persistent; 96 + 32 levels per step)"
+    sources = [CSRC + "bl_gemv_stream_mma.cuh", CSRC + "bl_gemv_stream.cuh", CSRC + "bl_gemv_mma.cuh",
+               CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
+    traffic_file = "gemv_w1a16_stream_mma_7b_decode_batch16.traffic.json"
+
+
+WORKLOADS = {w.name: w for w in (Decode, Prefill, Backward, W1A8, W1A8Single, W158A8, W1A8Tensor, W1A1,
+                                   DecodeStack, DecodeStack16)}
 
 
 # ----------------------------------------------------------------------------- ours
@@ -943,20 +1080,14 @@ def summarize(wl, ms, ms_e2e, steps, world, peaks, peak_kind):
 
 def secondary_llama7b(dev, peaks):
     """All 224 linears of a 7B-shaped model (0.8 GB of signs, more than L2):
-    decode at batch 1 and 16 as one dependent chain per token step
+    decode at batch 1 and 16 as a chain of 224 launches per token step
     (x -> q,k,v; v -> o; o -> gate,up; up -> down -> next layer), CUDA graph
-    of one step, and a 4096-token prefill."""
+    of one step, and a 4096-token prefill. The same chain as one stacked
+    call per step is the decode_stack / decode_stack16 workload."""
     import torch
     import bit_linear_layers_b200 as bl
     import synthetic
-    layers = []
-    for layer in range(synthetic.LLAMA7B_LAYERS):
-        mats = []
-        for idx, (K, N) in enumerate(synthetic.LLAMA7B_LAYER):
-            W = synthetic.weights(N, K, seed=5000 + 16 * layer + idx, device=dev)
-            mats.append(bl.bin_pack(W, bl.BL_PACK_FBI))
-            del W
-        layers.append(mats)
+    layers = llama7b_layers(dev)
     packed_bytes = sum(p.numel() * 4 for mats in layers for p, _ in mats)
     flags = bl.BL_FLAG_OVERLAP_PREVIOUS
     res = {"packed_GB": packed_bytes / 1e9}
@@ -1003,39 +1134,6 @@ def secondary_llama7b(dev, peaks):
                                    "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                    "launches_per_step": 224}
         del gph
-        # the same chain as one stacked call: 128 levels (q,k,v | o | gate,up | down per
-        # layer), every linear writing a buffer of its own
-        levels = []
-        cur = x.reshape(-1) if B == 1 else x
-        shp = (lambda n: (n,)) if B == 1 else (lambda n: (B, n))
-        for mats in layers:
-            lq, lk, lv, lo, lh = (torch.empty(shp(4096), dtype=torch.bfloat16, device=dev) for _ in range(5))
-            lg, lu = (torch.empty(shp(11008), dtype=torch.bfloat16, device=dev) for _ in range(2))
-            levels.append((cur, [(mats[0][0], mats[0][1], lq), (mats[1][0], mats[1][1], lk),
-                                 (mats[2][0], mats[2][1], lv)]))
-            levels.append((lv, [(mats[3][0], mats[3][1], lo)]))
-            levels.append((lo, [(mats[4][0], mats[4][1], lg), (mats[5][0], mats[5][1], lu)]))
-            levels.append((lu, [(mats[6][0], mats[6][1], lh)]))
-            cur = lh
-        stack = bl.W1A16Stack(levels)
-        for _ in range(3):
-            stack.run()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(reps):
-            stack.run()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / reps
-        res[f"decode_batch{B}_stack"] = {
-            "ms_per_token_step": ms, "tok_s": B / (ms * 1e-3),
-            "packed_GB_per_s": packed_bytes / (ms * 1e-3) / 1e9,
-            "hbm_frac": packed_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "launches_per_step": 3, "call": "bin_linear_w1a16_stack_batch (one zero-fill of the tagged outputs + "
-                                             "two persistent kernels)"}
-        del stack, levels
     # prefill: 4096 tokens through every linear (not chained: fixed inputs)
     T = 4096
     x4 = synthetic.activations(T, 4096, seed=78, device=dev)
@@ -1287,6 +1385,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = WORKLOADS[args.workload]()
+    wl_metric, wl_unit, wl_dtype, wl_launches = wl.metric, wl.unit, wl.dtype, wl.launches_per_step
     config = dict(wl.config)
     config["timing"] = ("K steps in one CUDA graph, timed by CUDA events recorded as the graph's first and last "
                         "nodes (the launching stream)")
@@ -1336,11 +1435,11 @@ def main():
         torch.cuda.empty_cache()
         extra = secondary(args, dev, peaks, peak_kind)
     line = {
-        "metric": WORKLOADS[args.workload].metric, "value": value, "unit": roof["unit"], "n_gpus": world,
+        "metric": wl_metric, "value": value, "unit": wl_unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": WORKLOADS[args.workload].dtype, "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": wl_dtype, "data": "synthetic",
         "config": config, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": args.steps * WORKLOADS[args.workload].launches_per_step,
+        "gpu_launches": args.steps * wl_launches,
         "clocks": clocks, "secondary": extra,
     }
     print(json.dumps(line), flush=True)

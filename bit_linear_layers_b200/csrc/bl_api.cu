@@ -103,10 +103,10 @@ int device_setup(int* num_sms) {
     if (!ok) cudaGetLastError();
     {
       // how many clusters of 8 of a stack kernel can be resident at once
-      auto stack_capacity = [](auto kernel, int smem) {
+      auto stack_capacity = [](auto kernel, int threads, int smem) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(kStrCluster, 1, 1);
-        cfg.blockDim = dim3(kStrThreads + 32, 1, 1);
+        cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
         cfg.dynamicSmemBytes = static_cast<size_t>(smem);
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -122,9 +122,9 @@ int device_setup(int* num_sms) {
         }
         return n;
       };
-      st.stack_clusters = stack_capacity(gemv_w1a16_stream_kernel, kStrSmemBytes);
-      st.stack_mma_clusters[0] = stack_capacity(gemv_w1a16_stream_mma_kernel<8>, SmCfg<8>::kSmemBytes);
-      st.stack_mma_clusters[1] = stack_capacity(gemv_w1a16_stream_mma_kernel<16>, SmCfg<16>::kSmemBytes);
+      st.stack_clusters = stack_capacity(gemv_w1a16_stream_kernel, kStrThreads + 32, kStrSmemBytes);
+      st.stack_mma_clusters[0] = stack_capacity(gemv_w1a16_stream_mma_kernel<8>, kSmThreads + 32, SmCfg<8>::kSmemBytes);
+      st.stack_mma_clusters[1] = stack_capacity(gemv_w1a16_stream_mma_kernel<16>, kSmThreads + 32, SmCfg<16>::kSmemBytes);
     }
     for (int S : {2, 4, 8}) {
       cudaLaunchConfig_t cfg = {};
@@ -217,7 +217,7 @@ int check_shape(int64_t M, int64_t N, int64_t K) {
   return BL_OK;
 }
 
-// ---- few-token warp-MMA GEMV (5 <= M <= 16, K % 256 == 0, K <= 12288) ---------------
+// ---- few-token warp-MMA GEMV (2 <= M <= 16, K % 256 == 0, K <= 12288) ---------------
 template <int MT, int SWMAX>
 cudaError_t launch_mma_t(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y, int M,
                          int N, int K, bool overlap, cudaStream_t s) {
@@ -600,7 +600,7 @@ int bin_linear_w1a16_ex(const uint16_t* x, const uint32_t* packed, const float* 
     }
     return launch_status();
   }
-  if (M > 4 && M <= 16 && K % 256 == 0 && K / 256 <= kMmaMaxSliceWords) {  // measured faster than tcgen05 here
+  if (M > 1 && M <= 16 && K % 256 == 0 && K / 256 <= kMmaMaxSliceWords) {  // measured faster than tcgen05 here
     const cudaError_t e = launch_mma(x, packed, alpha, y, int(M), int(N), int(K),
                                      (flags & BL_FLAG_OVERLAP_PREVIOUS) != 0, s);
     if (e != cudaSuccess) {
@@ -779,7 +779,7 @@ int bin_linear_w1a16_stack_batch(const bl_stack_level* levels, int num_levels, c
     const int clusters = int(max_chunks < G ? max_chunks : G);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kStrCluster, static_cast<unsigned>(clusters), 1);
-    cfg.blockDim = dim3(kStrThreads + 32, 1, 1);
+    cfg.blockDim = dim3(M == 1 ? kStrThreads + 32 : kSmThreads + 32, 1, 1);
     cfg.dynamicSmemBytes = M == 1 ? kStrSmemBytes : (M <= 8 ? SmCfg<8>::kSmemBytes : SmCfg<16>::kSmemBytes);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

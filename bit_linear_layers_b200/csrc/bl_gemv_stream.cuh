@@ -49,7 +49,10 @@
 //
 // Partial sums. After a pass, each row's slice partial goes to the row's
 // owner in the cluster (st.async into inbox buffer n % 2 of pass n, counted
-// on that buffer's inbox_full barrier). No CTA can overwrite a buffer that is
+// on that buffer's inbox_full barrier). With the partials every CTA also
+// sends each peer (itself included) a 4-byte token on the same barrier, so a
+// pass's inbox fills only once every peer has pushed that pass, even for a
+// CTA that owns no live row of it. No CTA can overwrite a buffer that is
 // still being read: a CTA pushes pass n + 2 only after its own pass n + 1
 // inbox has filled, i.e. after every peer has pushed pass n + 1, which each
 // peer does only once its owners have read its pass n inbox (a barrier of the
@@ -129,8 +132,9 @@ __device__ __forceinline__ void cluster_arrive_release() {
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+template <int NTHREADS = kStrThreads>
 __device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kStrThreads) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(NTHREADS) : "memory");
 }
 
 // this CTA's slice window of a level with K inputs
@@ -196,7 +200,7 @@ __device__ __forceinline__ bool str_next_slab(const StrJob* jobs, const StrLevel
 // each slot reused once the compute warps have released it. Afterwards it
 // waits (bounded) for the last use of every slot, so that no copy is in
 // flight when the CTA exits.
-template <int PASS>
+template <int PASS, int SLOTS = kStrSlots>
 __device__ __forceinline__ void str_produce(const StrParams& P, const StrLevel* lvs, const StrJob* jobs,
                                             int num_levels, int cid, int G, uint32_t rank, uint8_t* ring,
                                             uint64_t* full, uint64_t* empty) {
@@ -215,9 +219,9 @@ __device__ __forceinline__ void str_produce(const StrParams& P, const StrLevel* 
       if (npass == 0) break;
       for (int pg = 0; pg < np; ++pg) {
         for (int i = 0; i < npass; ++i) {
-          const uint32_t slot = issued % kStrSlots;
-          if (issued >= static_cast<uint32_t>(kStrSlots) && live &&
-              !mbar_wait(smem_u32(&empty[slot]), ((issued / kStrSlots) - 1) & 1u, kWhereStackRing)) {
+          const uint32_t slot = issued % SLOTS;
+          if (issued >= static_cast<uint32_t>(SLOTS) && live &&
+              !mbar_wait(smem_u32(&empty[slot]), ((issued / SLOTS) - 1) & 1u, kWhereStackRing)) {
             st_relaxed_gpu_u32(P.abort, 1u);
             live = false;  // stop waiting; the outputs are undefined from here on
           }
@@ -233,9 +237,9 @@ __device__ __forceinline__ void str_produce(const StrParams& P, const StrLevel* 
       }
     }
   }
-  const uint32_t first = issued > static_cast<uint32_t>(kStrSlots) ? issued - kStrSlots : 0u;
+  const uint32_t first = issued > static_cast<uint32_t>(SLOTS) ? issued - SLOTS : 0u;
   for (uint32_t k = first; k < issued; ++k)
-    if (!mbar_wait(smem_u32(&full[k % kStrSlots]), (k / kStrSlots) & 1u, kWhereStackRing)) break;
+    if (!mbar_wait(smem_u32(&full[k % SLOTS]), (k / SLOTS) & 1u, kWhereStackRing)) break;
 }
 
 // Warps 0..15 compute (kStrThreads threads); warp 16 streams the weights.
@@ -247,7 +251,8 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_kernel(
   uint16_t* xs = reinterpret_cast<uint16_t*>(ring + kStrSlots * kStrSlotBytes);  // window inputs
   __shared__ float inbox[2][kStrPass * kStrRows];       // [pass % 2][slab of the pass][source rank][owned row]
   static_assert(kStrThreads >= kStrPass * kStrRows / kStrCluster, "one owner thread per owned row of a pass");
-  __shared__ __align__(8) uint64_t inbox_full[2];       // a pass's partials have all landed (bytes)
+  __shared__ __align__(8) uint64_t inbox_full[2];       // a pass's partials and tokens have all landed (bytes)
+  __shared__ float tokens[2][kStrCluster];              // [pass % 2][source rank]
   __shared__ __align__(8) uint64_t full[kStrSlots];     // a slot's tensor copies have landed
   __shared__ __align__(8) uint64_t empty[kStrSlots];    // every compute warp is done with a slot
   // the level and linear descriptors, read many times: kept in shared memory
@@ -344,14 +349,15 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_kernel(
         for (int i = 0; i < kStrPass; ++i)
           if (npass == i && str_next_slab(jobs, lv, run, sl[i])) ++npass;
         if (npass == 0) break;
-        // bytes of partials this CTA will receive: 8 ranks x 4 bytes per owned live row
+        // bytes this CTA will receive: 8 ranks x 4 bytes per owned live row,
+        // and one 4-byte token from each rank
         if (tid == 0) {
           uint32_t rows = 0;
           for (int i = 0; i < npass; ++i) {
             const int r = sl[i].nc() * kStrChunk - static_cast<int>(rank) * kOwned;
             rows += r <= 0 ? 0u : (r >= kOwned ? static_cast<uint32_t>(kOwned) : static_cast<uint32_t>(r));
           }
-          mbar_arrive_expect_tx(smem_u32(&inbox_full[n & 1u]), rows * kStrCluster * 4);
+          mbar_arrive_expect_tx(smem_u32(&inbox_full[n & 1u]), (rows + 1) * kStrCluster * 4);
         }
         // owners: thread t will add the 8 partials of row t % 32 of slab t / 32;
         // its scale is read now, off the critical path
@@ -432,6 +438,11 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_kernel(
 #pragma unroll
           for (int i = 0; i < kStrPass; ++i)
             if (i < npass && warp < sl[i].nc()) st_async_f32(rslot + i * kStrRows * 4, part[i], rbar);
+        }
+        if (warp == 0 && lane < kStrCluster) {  // this pass's token to rank `lane`
+          const uint32_t dst = static_cast<uint32_t>(lane);
+          st_async_f32(map_to_rank(smem_u32(&tokens[n & 1u][rank]), dst), 0.f,
+                       map_to_rank(smem_u32(&inbox_full[n & 1u]), dst));
         }
         uint16_t* yp = nullptr;
         uint32_t* tp = nullptr;

@@ -118,9 +118,9 @@ int bin_pack(const float* W, int64_t N, int64_t K, int mode, uint32_t* packed, f
  * only initialises them), y [M x N] bf16 (round to nearest even).
  * Accumulation is fp32. A single token uses a lookup-table GEMV (a cluster
  * of CTAs splits K; signed byte sums of x are tabulated in shared memory);
- * up to 4 tokens a predicated-add GEMV; 5 to 16 tokens (K % 256 == 0,
- * K <= 12288) a GEMV whose products run on the warp-level MMA; more tokens a
- * tcgen05 tensor-core GEMM. No workspace.
+ * 2 to 16 tokens with K % 256 == 0 and K <= 12288 a GEMV whose products run
+ * on the warp-level MMA; other shapes of up to 4 tokens a predicated-add
+ * GEMV; more tokens a tcgen05 tensor-core GEMM. No workspace.
  */
 int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alpha, uint16_t* y,
                      int64_t M, int64_t N, int64_t K, void* stream);
@@ -129,10 +129,10 @@ int bin_linear_w1a16(const uint16_t* x, const uint32_t* packed, const float* alp
  * bin_linear_w1a16_ex -- bin_linear_w1a16 with launch flags.
  *   BL_FLAG_OVERLAP_PREVIOUS: the caller promises that `packed` and `alpha`
  *   are not written by the kernel enqueued immediately before this call on
- *   `stream` (true for a chain of inference layers). The single-token kernel
- *   may then start streaming the weights before that kernel has finished
- *   (programmatic dependent launch); it still waits for it before reading x
- *   or writing y. Other kernels ignore the flag. flags = 0 is exactly
+ *   `stream` (true for a chain of inference layers). The lookup-table and
+ *   warp-MMA GEMVs (1 to 16 tokens) may then start streaming the weights
+ *   before that kernel has finished (programmatic dependent launch); they
+ *   still wait for it before reading x or writing y. Other kernels ignore the flag. flags = 0 is exactly
  *   bin_linear_w1a16.
  */
 #define BL_FLAG_OVERLAP_PREVIOUS 1u

@@ -40,11 +40,11 @@ FULL = [
     # ragged row clusters, and K with no split (falls back to the predicated GEMV)
     (1, 128, 128), (1, 4096, 4096), (1, 1000, 11008), (1, 257, 2048), (1, 300, 640), (1, 513, 5632),
     (1, 4099, 384), (1, 77, 8320),
-    # few-token GEMV path (M <= 4)
-    (2, 300, 384), (3, 129, 256), (4, 1000, 11008),
-    # 5..16 tokens, K % 256 == 0: warp-MMA GEMV (8- and 16-token tiles, 16- and 48-word slices,
+    # 2..4 tokens with K % 256 != 0: predicated-add GEMV
+    (2, 300, 384), (4, 129, 640),
+    # 2..16 tokens, K % 256 == 0: warp-MMA GEMV (8- and 16-token tiles, 16- and 48-word slices,
     # slices shorter than a word group, ragged row clusters)
-    (6, 384, 256), (8, 1000, 4096), (9, 129, 2048), (12, 4099, 512), (16, 300, 4096), (16, 257, 11008),
+    (2, 1000, 4096), (3, 129, 256), (4, 1000, 11008), (4, 4099, 512), (6, 384, 256), (8, 1000, 4096), (9, 129, 2048), (12, 4099, 512), (16, 300, 4096), (16, 257, 11008),
     (7, 200, 12288), (13, 128, 8192),
     # tcgen05 GEMM path
     (5, 384, 384), (16, 128, 128), (17, 200, 384), (129, 383, 640), (256, 512, 1024),

@@ -9,7 +9,8 @@ layers in one persistent launch) on the GPU.
   also splits K eight ways (K = 4096 and 11008, the 7B shapes);
 * decode batches of 2..16 tokens (bin_linear_w1a16_stack_batch): every token
   of every level against the oracle, at small and 7B shapes;
-* stacks longer than one launch (more than 96 levels or 144 linears);
+* stacks longer than one launch (more than 96 levels or 144 linears), at
+  one token and in batches;
 * the argument checks."""
 import ctypes
 
@@ -178,6 +179,46 @@ def test_stack_many_linears_per_launch(bl, oracle):
     assert bl.device_error() == (0, 0)
     for i in range(3):
         _check_level(oracle, xs[i], [(packed, alpha, y) for y in ys[i][::33]], f"level {i}")
+
+
+@pytest.mark.parametrize("M", [3, 16])
+def test_stack_batch_many_small_linears(bl, oracle, M):
+    """300 linears of 64 rows over 3 levels: every slab is one linear's 4
+    chunks, paired into passes; more linears than one launch takes."""
+    import synthetic
+    K = 256
+    dp, da, packed, alpha = _linear(oracle, 64, K, 92)
+    xs = [synthetic.activations(M, K, 93 + i).cuda() for i in range(3)]
+    ys = [[torch.empty((M, 64), dtype=torch.bfloat16, device="cuda") for _ in range(100)] for _ in range(3)]
+    levels = [(xs[i], [(dp, da, y) for y in ys[i]]) for i in range(3)]
+    bl.W1A16Stack(levels).run()
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
+    for i in range(3):
+        _check_level(oracle, xs[i], [(packed, alpha, y) for y in ys[i][::11]], f"level {i}")
+
+
+def test_stack_batch_longer_than_one_launch(bl, oracle):
+    """110 chained levels at 5 tokens (two launches), alternating K = 512 and 768."""
+    import synthetic
+    M = 5
+    mats = {(K, N): _linear(oracle, N, K, 70 + K // 256) for K, N in [(512, 768), (768, 512)]}
+    x0 = synthetic.activations(M, 512, 79).cuda()
+    levels, cur, outs = [], x0, []
+    for i in range(110):
+        K, N = (512, 768) if i % 2 == 0 else (768, 512)
+        dp, da, _, _ = mats[(K, N)]
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        levels.append((cur, [(dp, da, y)]))
+        outs.append((cur, (K, N), y))
+        cur = y
+    bl.W1A16Stack(levels).run()
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
+    for i in (0, 1, 94, 95, 96, 97, 109):
+        x, KN, y = outs[i]
+        _, _, packed, alpha = mats[KN]
+        _check_level(oracle, x, [(packed, alpha, y)], f"level {i}")
 
 
 def test_stack_argument_checks(bl):
