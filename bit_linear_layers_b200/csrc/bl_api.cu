@@ -96,6 +96,7 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_stream_mma_kernel<8>, SmCfg<8>::kSmemBytes) &&
               set_smem(gemv_w1a16_stream_mma_kernel<16>, SmCfg<16>::kSmemBytes) &&
               set_smem(gemm_ss_ste_kernel, kSsSmemBytes) &&
+              set_smem(transpose_pack_dup_kernel, kTpSmemBytes) &&
               set_smem(gemv_w1a16_mma_kernel<8, 16>, mma_smem_bytes(8, 16)) &&
               set_smem(gemv_w1a16_mma_kernel<16, 16>, mma_smem_bytes(16, 16)) &&
               set_smem(gemv_w1a16_mma_kernel<8, kMmaMaxSliceWords>, mma_smem_bytes(8, kMmaMaxSliceWords)) &&
@@ -840,14 +841,13 @@ int bin_linear_w1a16_backward(const uint16_t* x, const uint32_t* packed, const f
   auto* dyt = reinterpret_cast<uint16_t*>(w);
   w += align256(size_t(N) * size_t(Mp) * 2);
   auto* part = reinterpret_cast<float*>(w);  // [K / 128][N] signed partial sums for dalpha
-  const unsigned ew_grid = static_cast<unsigned>(sms * 8);
   if (dx) {
     // dx = [hi | lo] x [S^T | S^T] through the forward path (unit scales)
-    ste_scale_split_kernel<<<ew_grid, 256, 0, s>>>(dy, alpha, M, N, g2);
+    ste_scale_split_kernel<<<dim3(static_cast<unsigned>(cdiv(N / 8, 256)), static_cast<unsigned>(M < 8192 ? M : 8192)),
+                             256, 0, s>>>(dy, alpha, M, N, g2);
     if ((rc = launch_status()) != BL_OK) return rc;
-    const int64_t warps = (N / 32) * (K / 32);
-    const int64_t blocks = cdiv(warps, 8) < int64_t(sms) * 16 ? cdiv(warps, 8) : int64_t(sms) * 16;
-    transpose_pack_dup_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(packed, N, K, packed_t2);
+    transpose_pack_dup_kernel<<<dim3(static_cast<unsigned>(cdiv(N, kTpRows)), static_cast<unsigned>(cdiv(K / 32, kTpWords))),
+                                256, kTpSmemBytes, s>>>(packed, N, K, packed_t2);
     if ((rc = launch_status()) != BL_OK) return rc;
     fill_f32_kernel<<<static_cast<unsigned>(cdiv(K, 256) < sms ? cdiv(K, 256) : sms), 256, 0, s>>>(ones, K, 1.0f);
     if ((rc = launch_status()) != BL_OK) return rc;
@@ -857,9 +857,9 @@ int bin_linear_w1a16_backward(const uint16_t* x, const uint32_t* packed, const f
   if (dw) {
     // P = dY^T X on the tensor cores, then dW = alpha P and dalpha = sum_k s P in place
     const dim3 tb(32, 8);
-    transpose_bf16_kernel<<<dim3(unsigned(cdiv(K, 32)), unsigned(cdiv(Mp, 32))), tb, 0, s>>>(x, M, K, xt, Mp);
+    transpose_bf16_kernel<<<dim3(unsigned(K / kTrTile), unsigned(Mp / kTrTile)), tb, 0, s>>>(x, M, K, xt, Mp);
     if ((rc = launch_status()) != BL_OK) return rc;
-    transpose_bf16_kernel<<<dim3(unsigned(cdiv(N, 32)), unsigned(cdiv(Mp, 32))), tb, 0, s>>>(dy, M, N, dyt, Mp);
+    transpose_bf16_kernel<<<dim3(unsigned(N / kTrTile), unsigned(Mp / kTrTile)), tb, 0, s>>>(dy, M, N, dyt, Mp);
     if ((rc = launch_status()) != BL_OK) return rc;
     CUtensorMap tm_a, tm_b;
     if (!make_map_2d(&tm_a, xt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(Mp), uint64_t(K), kSsUnit, kSsRowsA,

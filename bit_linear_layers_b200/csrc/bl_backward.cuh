@@ -27,63 +27,129 @@ namespace bl {
 // ---- element-wise and layout kernels -----------------------------------------------
 
 // g = dy * alpha_j in fp32, split into bf16 hi (round to nearest) and bf16 lo
-// = the rounding of the remainder: row m of g2 is [hi_m0..hi_mN-1 | lo_m0..lo_mN-1]
+// = the rounding of the remainder: row m of g2 is [hi_m0..hi_mN-1 | lo_m0..lo_mN-1].
+// Each thread takes 8 consecutive outputs of a row (16-byte loads of dy and
+// stores of g2); rows are spread over grid y. N % 8 == 0, 16-byte aligned rows.
 __global__ void ste_scale_split_kernel(const uint16_t* __restrict__ dy, const float* __restrict__ alpha, int64_t M,
                                        int64_t N, uint16_t* __restrict__ g2) {
-  const int64_t total = M * N;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t m = i / N, j = i - m * N;
-    const float g = bf16_bits_to_float(dy[i]) * alpha[j];
-    const uint16_t hi = float_to_bf16_bits(g);
-    const uint16_t lo = float_to_bf16_bits(g - bf16_bits_to_float(hi));
-    g2[m * 2 * N + j] = hi;
-    g2[m * 2 * N + N + j] = lo;
+  const int64_t groups = N / 8;
+  for (int64_t m = blockIdx.y; m < M; m += gridDim.y) {
+    const uint4* drow = reinterpret_cast<const uint4*>(dy + m * N);
+    uint4* hrow = reinterpret_cast<uint4*>(g2 + m * 2 * N);
+    uint4* lrow = reinterpret_cast<uint4*>(g2 + m * 2 * N + N);
+    for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < groups;
+         q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const uint4 d = drow[q];
+      const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
+      float av[8];  // (alpha need not be 16-byte aligned)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) av[e] = alpha[8 * q + e];
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t h2 = 0u, l2 = 0u;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float g = bf16_bits_to_float(static_cast<uint16_t>(dw[i] >> (16 * e))) * av[2 * i + e];
+          const uint16_t hi = float_to_bf16_bits(g);
+          const uint16_t lo = float_to_bf16_bits(g - bf16_bits_to_float(hi));
+          h2 |= static_cast<uint32_t>(hi) << (16 * e);
+          l2 |= static_cast<uint32_t>(lo) << (16 * e);
+        }
+        hw[i] = h2;
+        lw[i] = l2;
+      }
+      hrow[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      lrow[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
   }
 }
 
 // Packed signs [N][K/32] -> their transpose [K][2N/32], each row written
-// twice (words 0..N/32-1 and again N/32..2N/32-1). One warp per 32 x 32 bit
-// block: lane l holds word (row j0 + l, column word kw); the ballot of bit b
-// over the lanes is word j0/32 of transposed row 32 kw + b. N % 32 == 0.
-__global__ void transpose_pack_dup_kernel(const uint32_t* __restrict__ packed, int64_t N, int64_t K,
-                                          uint32_t* __restrict__ out) {
-  const int64_t nw = N / 32, kw_count = K / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; wid < nw * kw_count;
-       wid += warps) {
-    const int64_t jb = wid / kw_count, kw = wid - jb * kw_count;
-    const uint32_t w = packed[(jb * 32 + lane) * kw_count + kw];
-    uint32_t mine = 0u;
+// twice (words 0..N/32-1 and again N/32..2N/32-1). A CTA takes 256 rows j
+// (8 output words) by 256 k (8 input words): the rows' words are read into
+// shared memory (32 bytes per row), each warp turns 32 x 32 bit blocks
+// around in registers, and the output rows leave as 32-byte segments. The
+// block transpose: lane l holds row l (bit c = column c); five exchange
+// stages with the lane l ^ s (s = 16, 8, 4, 2, 1) swap the off-diagonal s x s
+// sub-blocks of every 2s x 2s block, after which lane c holds column c (bit
+// l = row l). N % 128 == 0 (a ragged last tile of rows reads zeros past N),
+// K % 128 == 0.
+constexpr int kTpRows = 256;                 // rows j per tile (8 output words)
+constexpr int kTpWords = 8;                  // input words per row per tile (256 k)
+constexpr int kTpInPitch = kTpWords + 1;     // words: a block's column reads hit 32 banks
+constexpr int kTpOutWords = kTpRows / 32;    // 8
+constexpr int kTpSmemBytes = (kTpRows * kTpInPitch + kTpWords * 32 * kTpOutWords) * 4;
+__device__ __forceinline__ uint32_t transpose32_warp(uint32_t x, int lane) {
 #pragma unroll
-    for (int b = 0; b < 32; ++b) {
-      const uint32_t col = __ballot_sync(0xffffffffu, (w >> b) & 1u);
-      if (lane == b) mine = col;
-    }
-    uint32_t* row = out + (kw * 32 + lane) * 2 * nw;
-    row[jb] = mine;
-    row[nw + jb] = mine;
+  for (int s = 16; s >= 1; s >>= 1) {
+    const uint32_t m = s == 16 ? 0x0000FFFFu : s == 8 ? 0x00FF00FFu : s == 4 ? 0x0F0F0F0Fu : s == 2 ? 0x33333333u
+                                                                                                     : 0x55555555u;
+    const uint32_t t = __shfl_xor_sync(0xffffffffu, x, s);
+    x = (lane & s) ? ((x & ~m) | ((t & ~m) >> s)) : ((x & m) | ((t & m) << s));
+  }
+  return x;
+}
+__global__ void __launch_bounds__(256) transpose_pack_dup_kernel(const uint32_t* __restrict__ packed, int64_t N,
+                                                                 int64_t K, uint32_t* __restrict__ out) {
+  extern __shared__ uint32_t tp_smem[];
+  uint32_t* in_t = tp_smem;                            // [256 rows][9]
+  uint32_t* out_t = tp_smem + kTpRows * kTpInPitch;   // [8 kw x 32 b][8 words]
+  const int64_t nw = N / 32, kw_count = K / 32;
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * kTpRows;
+  const int64_t kw0 = static_cast<int64_t>(blockIdx.y) * kTpWords;  // K % 256 need not hold: kws may be 4
+  const int kws = static_cast<int>(kw_count - kw0 < kTpWords ? kw_count - kw0 : kTpWords);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < kTpRows * kTpWords; e += 256) {
+    const int r = e / kTpWords, c = e % kTpWords;
+    in_t[r * kTpInPitch + c] = (c < kws && j0 + r < N) ? packed[(j0 + r) * kw_count + kw0 + c] : 0u;
+  }
+  __syncthreads();
+  // block (jb, kw): rows 32 jb .. + 31 of the tile, word kw; warp w takes jb = w
+  for (int kw = 0; kw < kws; ++kw) {
+    const uint32_t col = transpose32_warp(in_t[(32 * warp + lane) * kTpInPitch + kw], lane);
+    out_t[(kw * 32 + lane) * kTpOutWords + warp] = col;  // output row 32 (kw0 + kw) + lane, word j0 / 32 + warp
+  }
+  __syncthreads();
+  // output rows 32 kw0 .. + 32 kws - 1: 8 words (two 16-byte stores) at column j0 / 32, twice
+  const int64_t jw0 = j0 / 32;
+  const int jws = static_cast<int>(nw - jw0 < kTpOutWords ? nw - jw0 : kTpOutWords);  // 4 or 8
+  for (int e = tid; e < kws * 32 * 2; e += 256) {
+    const int orow = e >> 1, half = e & 1;
+    if (4 * half >= jws) continue;
+    const uint32_t* src = out_t + orow * kTpOutWords + 4 * half;
+    uint32_t* dst = out + (32 * kw0 + orow) * 2 * nw + jw0 + 4 * half;
+    const uint4 v = make_uint4(src[0], src[1], src[2], src[3]);
+    *reinterpret_cast<uint4*>(dst) = v;
+    *reinterpret_cast<uint4*>(dst + nw) = v;
   }
 }
 
-// bf16 [R][C] -> [C][Rp] (Rp >= R; entries r >= R are zero): 32 x 32 tiles
-// through shared memory, block (32, 8)
+// bf16 [R][C] -> [C][Rp] (Rp >= R; entries r >= R are zero): 64 x 64 tiles
+// through shared memory, block (32, 8), pairs of elements per access (a
+// warp reads or writes 128 contiguous bytes). C % 64 == 0, Rp % 64 == 0,
+// 4-byte aligned rows.
+constexpr int kTrTile = 64;
+constexpr int kTrPitch = kTrTile + 2;  // halfwords: rows 4-byte aligned, pair stores conflict-free
 __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int64_t R, int64_t C,
                                       uint16_t* __restrict__ out, int64_t Rp) {
-  __shared__ uint16_t tile[32][33];
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 32, r0 = static_cast<int64_t>(blockIdx.y) * 32;
+  __shared__ __align__(4) uint16_t tile[kTrTile][kTrPitch];
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTrTile, r0 = static_cast<int64_t>(blockIdx.y) * kTrTile;
   const int tx = threadIdx.x, ty = threadIdx.y;
+  // rows r0 + ty + 8 i, columns c0 + 2 tx and + 1
 #pragma unroll
-  for (int i = 0; i < 32; i += 8) {
-    const int64_t r = r0 + ty + i, c = c0 + tx;
-    tile[ty + i][tx] = (r < R && c < C) ? in[r * C + c] : static_cast<uint16_t>(0);
+  for (int i = 0; i < kTrTile; i += 8) {
+    const int64_t r = r0 + ty + i;
+    const uint32_t v = r < R ? *reinterpret_cast<const uint32_t*>(in + r * C + c0 + 2 * tx) : 0u;
+    *reinterpret_cast<uint32_t*>(&tile[ty + i][2 * tx]) = v;
   }
   __syncthreads();
+  // output rows c0 + ty + 8 i, elements r0 + 2 tx and + 1
 #pragma unroll
-  for (int i = 0; i < 32; i += 8) {
-    const int64_t c = c0 + ty + i, r = r0 + tx;
-    if (c < C && r < Rp) out[c * Rp + r] = tile[tx][ty + i];
+  for (int i = 0; i < kTrTile; i += 8) {
+    const int cc = ty + i;
+    const uint32_t v = static_cast<uint32_t>(tile[2 * tx][cc]) | (static_cast<uint32_t>(tile[2 * tx + 1][cc]) << 16);
+    *reinterpret_cast<uint32_t*>(out + (c0 + cc) * Rp + r0 + 2 * tx) = v;
   }
 }
 

@@ -39,7 +39,7 @@ def _check(got, ref, bound, what):
 
 
 FULL = [(1, 128, 128), (3, 256, 384), (17, 384, 256), (64, 128, 640), (100, 640, 512), (300, 256, 1024),
-        (130, 1024, 256)]
+        (130, 1024, 256), (5, 384, 1152)]
 
 
 @pytest.mark.parametrize("M,N,K", FULL)
