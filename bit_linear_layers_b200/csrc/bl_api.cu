@@ -22,6 +22,7 @@
 #include "bl_gemv_mma.cuh"
 #include "bl_gemv_stream.cuh"
 #include "bl_gemv_stream_mma.cuh"
+#include "bl_gemv_w1a8_mma.cuh"
 #include "bl_lnquant.cuh"
 #include "bl_pack.cuh"
 #include "bl_xnor.cuh"
@@ -97,6 +98,10 @@ int device_setup(int* num_sms) {
               set_smem(gemv_w1a16_stream_mma_kernel<16>, SmCfg<16>::kSmemBytes) &&
               set_smem(gemm_ss_ste_kernel, kSsSmemBytes) &&
               set_smem(transpose_pack_dup_kernel, kTpSmemBytes) &&
+              set_smem(gemv_w1a8_mma_kernel<8, false>, qm_smem_bytes(8, kQmMaxSliceWords, false)) &&
+              set_smem(gemv_w1a8_mma_kernel<16, false>, qm_smem_bytes(16, kQmMaxSliceWords, false)) &&
+              set_smem(gemv_w1a8_mma_kernel<8, true>, qm_smem_bytes(8, kQmMaxSliceWords, true)) &&
+              set_smem(gemv_w1a8_mma_kernel<16, true>, qm_smem_bytes(16, kQmMaxSliceWords, true)) &&
               set_smem(gemv_w1a16_mma_kernel<8, 16>, mma_smem_bytes(8, 16)) &&
               set_smem(gemv_w1a16_mma_kernel<16, 16>, mma_smem_bytes(16, 16)) &&
               set_smem(gemv_w1a16_mma_kernel<8, kMmaMaxSliceWords>, mma_smem_bytes(8, kMmaMaxSliceWords)) &&
@@ -455,9 +460,42 @@ int w1a8_impl(const uint16_t* x, const uint32_t* packed, const float* beta, floa
       cudaMemcpyAsync(gamma_out, gam, size_t(M) * sizeof(double), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return BL_ERR_CUDA;
 
+  if (M <= 16 && K % 256 == 0 && K / 256 <= kQmMaxSliceWords) {
+    // warp-level int8 MMA GEMV, a cluster of 8 CTAs per 64 rows; launched with
+    // programmatic serialisation (its weight copies start while the LN kernel
+    // runs; it waits for the codes before reading them)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kMmaCluster, static_cast<unsigned>(cdiv(N, kQmRows)), 1);
+    cfg.blockDim = dim3(kQmThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(qm_smem_bytes(M <= 8 ? 8 : 16, int(K / 256), ternary));
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kMmaCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const int m = int(M), n = int(N), k = int(K);
+    cudaError_t e;
+    if (ternary)
+      e = M <= 8 ? cudaLaunchKernelEx(&cfg, gemv_w1a8_mma_kernel<8, true>, codes, gam, packed, beta, y, acc_out, m, n, k)
+                 : cudaLaunchKernelEx(&cfg, gemv_w1a8_mma_kernel<16, true>, codes, gam, packed, beta, y, acc_out, m, n, k);
+    else
+      e = M <= 8 ? cudaLaunchKernelEx(&cfg, gemv_w1a8_mma_kernel<8, false>, codes, gam, packed, beta, y, acc_out, m, n, k)
+                 : cudaLaunchKernelEx(&cfg, gemv_w1a8_mma_kernel<16, false>, codes, gam, packed, beta, y, acc_out, m, n, k);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return BL_ERR_CUDA;
+    }
+    return launch_status();
+  }
   if (M <= 16) {
-    // launched with programmatic serialisation: scheduled while the LN kernel
-    // runs, it waits for that kernel's codes before reading them
+    // dp4a GEMV (K outside the MMA kernel's range), launched with programmatic
+    // serialisation: scheduled while the LN kernel runs, it waits for that
+    // kernel's codes before reading them
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(cdiv(N, kGemvRowsPerCta)), 1, 1);
     cfg.blockDim = dim3(kGemvThreads, 1, 1);

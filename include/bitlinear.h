@@ -228,6 +228,10 @@ int bin_linear_w1a16_stack_batch(const bl_stack_level* levels, int num_levels, c
  * pointer to one float (so pack -> forward needs no host round trip),
  * y [M x N] fp32. Needs ws of bl_workspace_bytes(BL_OP_W1A8, M, N, K) bytes
  * (the int8 codes and per-token gamma live there between the two kernels).
+ * Kernels: for M <= 16 with K <= 1024 and M * K <= 16384 one launch does
+ * everything; otherwise the LN + quantisation kernel, then for up to 16
+ * tokens a GEMV on the warp-level int8 MMA (K % 256 == 0, K <= 12288) or on
+ * dp4a (other K), for more tokens the tcgen05 int8 GEMM.
  */
 int bitlinear_w1a8(const uint16_t* x, const uint32_t* packed, const float* beta, float* y,
                    int64_t M, int64_t N, int64_t K, void* ws, size_t ws_bytes, void* stream);

@@ -73,7 +73,9 @@ def _run(bl, oracle, M, N, K, seed, full=True):
 # tiles split and unsplit, 128x256 tiles, ragged M and N
 FULL = [(1, 128, 128), (4, 256, 256), (7, 200, 384), (16, 129, 256), (17, 300, 512),
         (48, 700, 384), (130, 257, 640), (300, 1000, 1024), (20, 20000, 128), (100, 20000, 128),
-        (260, 9500, 128)]
+        (260, 9500, 128),
+        # warp-MMA GEMV (ternary planes, slices crossing 128-k blocks) and the dp4a GEMV
+        (1, 300, 2048), (5, 700, 5632), (16, 257, 12288), (9, 100, 1152)]
 
 
 @pytest.mark.parametrize("M,N,K", FULL)

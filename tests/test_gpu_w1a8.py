@@ -78,7 +78,11 @@ FULL = [(4, 256, 256), (1, 128, 128), (7, 200, 384), (16, 129, 256), (17, 300, 5
         # many tiles, ragged in M and N
         (260, 9500, 128),
         # 64-token tiles split along K; 32-, 64- and 128-token tiles with more tiles than SMs
-        (48, 700, 384), (20, 20000, 128), (40, 20000, 128), (100, 20000, 128)]
+        (48, 700, 384), (20, 20000, 128), (40, 20000, 128), (100, 20000, 128),
+        # decode batches past the one-launch path: the warp-MMA GEMV (K % 256 == 0, 1..16 tokens, slices
+        # of 8..48 words, ragged row clusters) and the dp4a GEMV (K % 256 != 0)
+        (1, 300, 2048), (4, 1000, 5632), (8, 64, 2048), (13, 513, 4096), (16, 5632, 2048), (16, 257, 12288),
+        (3, 100, 1152)]
 
 
 @pytest.mark.parametrize("M,N,K", FULL)

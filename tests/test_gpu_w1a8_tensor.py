@@ -80,7 +80,8 @@ def _run(bl, oracle, M, N, K, seed, mode, ternary, full=True, x=None):
 
 
 # decode GEMV (M <= 16), split and unsplit tensor-core tiles, ragged M and N
-FULL = [(1, 128, 128), (5, 200, 384), (16, 129, 256), (48, 700, 384), (130, 257, 640), (300, 1000, 1024)]
+FULL = [(1, 128, 128), (5, 200, 384), (16, 129, 256), (48, 700, 384), (130, 257, 640), (300, 1000, 1024),
+        (12, 300, 2048)]
 
 
 @pytest.mark.parametrize("ternary", [False, True], ids=["pm1", "ternary"])
