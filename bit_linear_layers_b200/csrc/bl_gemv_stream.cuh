@@ -49,14 +49,14 @@
 //
 // Partial sums. After a pass, each row's slice partial goes to the row's
 // owner in the cluster (st.async into inbox buffer n % 2 of pass n, counted
-// on that buffer's inbox_full barrier). With the partials every CTA also
-// sends each peer (itself included) a 4-byte token on the same barrier, so a
-// pass's inbox fills only once every peer has pushed that pass, even for a
-// CTA that owns no live row of it. No CTA can overwrite a buffer that is
-// still being read: a CTA pushes pass n + 2 only after its own pass n + 1
-// inbox has filled, i.e. after every peer has pushed pass n + 1, which each
-// peer does only once its owners have read its pass n inbox (a barrier of the
-// compute warps ends every pass).
+// on that buffer's inbox_full barrier). At the start of every pass each CTA
+// also sends each peer (itself included) a 4-byte token on that barrier: it
+// has read its inbox of the previous pass (a barrier of the compute warps
+// ends every pass). No CTA can overwrite a buffer that is still being read:
+// a CTA pushes pass n + 2 only after its own pass n + 1 inbox has filled,
+// which takes every peer's pass n + 1 token, which a peer sends only once it
+// has read its pass n inbox. (Without the tokens a CTA that owns no live row
+// of a pass would expect no bytes and nothing would hold it back.)
 //
 // Waits on weight slots, on input flags and on the partial-sum inbox are
 // bounded: past the limit the kernel records BL_ERR_TIMEOUT, sets the
@@ -359,6 +359,14 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_kernel(
           }
           mbar_arrive_expect_tx(smem_u32(&inbox_full[n & 1u]), (rows + 1) * kStrCluster * 4);
         }
+        // this pass's token to every rank: "done reading my pass n - 1 inbox"
+        // (true since the barrier that ended that pass), sent first so that it
+        // never holds up an inbox
+        if (warp == 0 && lane < kStrCluster) {
+          const uint32_t dst = static_cast<uint32_t>(lane);
+          st_async_f32(map_to_rank(smem_u32(&tokens[n & 1u][rank]), dst), 0.f,
+                       map_to_rank(smem_u32(&inbox_full[n & 1u]), dst));
+        }
         // owners: thread t will add the 8 partials of row t % 32 of slab t / 32;
         // its scale is read now, off the critical path
         const StrJob* ojb = nullptr;
@@ -438,11 +446,6 @@ __global__ void __launch_bounds__(kStrThreads + 32, 1) gemv_w1a16_stream_kernel(
 #pragma unroll
           for (int i = 0; i < kStrPass; ++i)
             if (i < npass && warp < sl[i].nc()) st_async_f32(rslot + i * kStrRows * 4, part[i], rbar);
-        }
-        if (warp == 0 && lane < kStrCluster) {  // this pass's token to rank `lane`
-          const uint32_t dst = static_cast<uint32_t>(lane);
-          st_async_f32(map_to_rank(smem_u32(&tokens[n & 1u][rank]), dst), 0.f,
-                       map_to_rank(smem_u32(&inbox_full[n & 1u]), dst));
         }
         uint16_t* yp = nullptr;
         uint32_t* tp = nullptr;
