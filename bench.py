@@ -189,7 +189,7 @@ class Workload:
             d = json.load(f)
         if d.get("src_hash") != src_hash(self.sources):
             return None
-        return d.get("dram_bytes_per_launch")
+        return d.get("dram_bytes_per_launch", d.get("dram_bytes_per_step"))
 
 
 class Decode(Workload):
@@ -853,9 +853,11 @@ class DecodeStack(Workload):
               "one stacked call per token step)")
     unit, scale, bound = "tok/s", 1.0, "hbm"
     roof_unit = "GB/s"
-    kernel = "gemv_w1a16_stream_kernel (15 clusters of 8 CTAs, persistent; 96 + 32 levels per step)"
+    kernel = ("gemv_w1a16_stream_kernel (15 clusters of 8 CTAs, persistent; two launches per step: 82 + 46 "
+              "levels, at most 144 linears per launch)")
     sources = [CSRC + "bl_gemv_stream.cuh", CSRC + "bl_gemv_lut.cuh", CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
     traffic_file = "gemv_w1a16_stream_7b_decode_batch1.traffic.json"
+    traffic_per = "step"  # achieved and traffic both cover the step's two launches
     launches_per_step = 2
 
     def __init__(self):
@@ -870,7 +872,8 @@ class DecodeStack(Workload):
                        "packed_bytes_per_step": self.packed_b, "algorithmic_bytes_per_step": self.alg_b,
                        "l2": f"inputs larger than L2: {self.packed_b / 1e6:.0f} MB of packed signs streamed per step",
                        "call": "bin_linear_w1a16_stack" + ("" if B == 1 else "_batch") +
-                               " (a zero-fill of the tagged outputs, then the persistent kernel per 96 levels)"}
+                               " (a zero-fill of the tagged outputs, then one persistent launch per 96 levels "
+                               "or 144 linears)"}
 
     def units_per_step(self):
         return float(self.B)  # tokens
@@ -941,7 +944,8 @@ class DecodeStack16(DecodeStack):
     B = 16
     metric = ("7B-shaped FBI-LLM linear-only decode tok/s at batch 16 (W1A16, 32 layers x 7 linears, "
               "one stacked call per token step)")
-    kernel = "gemv_w1a16_stream_mma_kernel<16> (15 clusters of 8 CTAs, persistent; 96 + 32 levels per step)"
+    kernel = ("gemv_w1a16_stream_mma_kernel<16> (15 clusters of 8 CTAs, persistent; two launches per step: "
+              "82 + 46 levels, at most 144 linears per launch)")
     sources = [CSRC + "bl_gemv_stream_mma.cuh", CSRC + "bl_gemv_stream.cuh", CSRC + "bl_gemv_mma.cuh",
                CSRC + "bl_common.cuh", CSRC + "bl_api.cu"]
     traffic_file = "gemv_w1a16_stream_mma_7b_decode_batch16.traffic.json"
@@ -1067,7 +1071,8 @@ def summarize(wl, ms, ms_e2e, steps, world, peaks, peak_kind):
     peak, peak_key = wl.peak(peaks, timed_s)
     achieved = wl.achieved(per_step_s)
     roof = {"bound": wl.bound, "achieved": achieved, "peak": peak, "unit": getattr(wl, "roof_unit", wl.unit),
-            "frac": achieved / peak, "traffic": wl.traffic(), "kernel": wl.kernel,
+            "frac": achieved / peak, "traffic": wl.traffic(), "traffic_per": getattr(wl, "traffic_per", "launch"),
+            "kernel": wl.kernel,
             "peak_source": peak_key if peak_key.startswith("derived")
             else (f"{peak_kind}: MEASURED_PEAKS.json {peak_key}" if peak_kind == "measured" else f"fallback ({peak_key})")}
     if isinstance(wl, Decode):
