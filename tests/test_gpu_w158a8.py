@@ -88,10 +88,12 @@ def test_w158a8_1p3b_sampled(bl, oracle, M, N, K):
     _run(bl, oracle, M, N, K, seed=5, full=False)
 
 
-def test_w158a8_unit_codes_give_plane_counts(bl):
+@pytest.mark.parametrize("M,K", [(40, 640), (7, 768)])
+def test_w158a8_unit_codes_give_plane_counts(bl, M, K):
     # codes all 1 (xq_in): acc_j = #(+1) - #(-1) of row j, from the planes
+    # (7 tokens, K % 256 == 0: the warp-MMA GEMV; 40 tokens: the GEMM)
     import synthetic
-    M, N, K = 40, 700, 640
+    N = 700
     W = synthetic.weights(N, K, 9, mean=0.001, device="cuda")
     packed, beta = bl.bin_pack(W, bl.BL_PACK_TERNARY)
     xq = torch.ones((M, K), dtype=torch.int8, device="cuda")

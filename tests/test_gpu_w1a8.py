@@ -123,8 +123,9 @@ def test_w1a8_constant_and_alternating_tokens(bl, oracle):
 
 def test_w1a8_unit_codes_give_popcount(bl):
     # with the quantisation bypassed and every code 1: acc_j = #pos - #neg
+    # (3 and 11 tokens: the warp-MMA GEMV's 8- and 16-token tiles; 150: the GEMM)
     import synthetic
-    for M in (3, 150):
+    for M in (3, 11, 150):
         N, K = 300, 512
         W = synthetic.weights(N, K, 8).cuda()
         packed, _, beta = bl.bin_pack(W, bl.BL_PACK_BITNET)
