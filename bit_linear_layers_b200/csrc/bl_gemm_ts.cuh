@@ -68,11 +68,14 @@ struct TsCfg {
   static constexpr int X_UNIT_BYTES = ATOMS * ATOM_BYTES;
   static constexpr int BITS_BYTES = ROWS * 16 * PLANES;         // one 128-k sign stage
   static constexpr int OUT_ELEM = KIND == 0 ? 2 : 4;            // y element bytes
-  // the output tile is staged in shared memory and written by bulk tensor
-  // stores: the whole tile at once when it fits in 64 KB, else one 128-row
-  // block at a time
+  // int8 tiles stage the fp32 output in shared memory and write it by bulk
+  // tensor stores (the whole tile at once when it fits in 64 KB, else one
+  // 128-row block at a time). bf16 tiles store straight from registers (each
+  // warp store is 64 contiguous bytes of a token row): the 64 KB a staging
+  // tile would take holds a third activation unit instead, and the mainloop
+  // waits on activation delivery (prefill 1049 -> 1217 TFLOP/s, measured)
   static constexpr int STAGE_COLS = ROWS * T * OUT_ELEM <= 64 * 1024 ? ROWS : 128;
-  static constexpr bool STAGE_OUT = !SPLIT && STAGE_COLS * T * OUT_ELEM <= 64 * 1024;
+  static constexpr bool STAGE_OUT = KIND != 0 && !SPLIT && STAGE_COLS * T * OUT_ELEM <= 64 * 1024;
   // split-K inbox rows: T partials padded by 16 bytes, so that a warp's
   // 16-byte reads of consecutive rows spread over all banks
   static constexpr int IN_STRIDE = T + 4;
@@ -608,12 +611,12 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
     }
   } else if (warp >= 4) {
     // ---------------- epilogue ----------------
-    // Accumulators -> scaled outputs -> staging tile [T tokens][STAGE_COLS]
-    // in shared memory -> one bulk tensor store per staged group of rows
-    // (rows/tokens past N/M are clipped by the store). The accumulators are
-    // released as soon as the last of them is read. Without an aligned
-    // output (N % 8 for bf16, N % 4 for fp32) the outputs are stored
-    // directly instead. The per-row alpha and per-token scale are read once
+    // Accumulators -> scaled outputs -> (int8 kinds) staging tile [T tokens]
+    // [STAGE_COLS] in shared memory -> one bulk tensor store per staged group
+    // of rows (rows/tokens past N/M are clipped by the store), or (bf16, and
+    // any unaligned output: N % 4 for fp32) stores straight to global memory,
+    // the range tests made once per 32-element chunk. The accumulators are
+    // released as soon as the last of them is read. The per-row alpha and per-token scale are read once
     // per tile into registers / shared memory, never per element.
     constexpr int BLK_PER_GROUP = C::STAGE_COLS / 128;
     const int q = warp & 3, et = threadIdx.x - 128;
@@ -675,11 +678,15 @@ __global__ void __launch_bounds__(kTsThreads, 1) gemm_ts_kernel(
                 const uint32_t so = smem_u32(stage_out) + (ml0 * C::STAGE_COLS + js) * 2;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) st_shared_u16(so + i * C::STAGE_COLS * 2, v[i]);
+              } else if (chunk_full) {
+                uint16_t* yp = reinterpret_cast<uint16_t*>(y) + static_cast<int64_t>(t0 + ml0) * N + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i, yp += N) *yp = v[i];
               } else if (jv) {
                 uint16_t* yp = reinterpret_cast<uint16_t*>(y) + static_cast<int64_t>(t0 + ml0) * N + j;
 #pragma unroll
                 for (int i = 0; i < 32; ++i, yp += N)
-                  if (chunk_full || t0 + ml0 + i < M) *yp = v[i];
+                  if (t0 + ml0 + i < M) *yp = v[i];
               }
             } else {
               // the fp32 form covers the chunk unless some |acc| is very large
