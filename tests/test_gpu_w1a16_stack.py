@@ -10,7 +10,8 @@ layers in one persistent launch) on the GPU.
 * decode batches of 2..16 tokens (bin_linear_w1a16_stack_batch): every token
   of every level against the oracle, at small and 7B shapes;
 * stacks longer than one launch (more than 96 levels or 144 linears), at
-  one token and in batches;
+  one token and in batches, including the full 7B-shaped chain the benchmark
+  times (sampled outputs across the launch boundary);
 * the argument checks."""
 import ctypes
 
@@ -18,7 +19,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity import bf16_to_f64, check_w1a16
+from parity import bf16_to_f64, check_w1a16, sample_positions
 
 pytestmark = pytest.mark.gpu
 
@@ -148,6 +149,50 @@ def test_stack_batch_at_7b_shapes(bl, oracle, M):
     words) at 8 and 16 tokens, every output against the oracle."""
     spec = [(4096, [4096, 512], None), (4096, [4096], (0, 0)), (4096, [11008], (1, 0)), (11008, [4096], (2, 0))]
     _run_and_check(bl, oracle, spec, seed0=60 + M, M=M)
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_stack_7b_full_chain_sampled(bl, oracle, M):
+    """The stacked decode exactly as the benchmark times it: all 224 linears of
+    a 7B-shaped model (32 layers; the same seeded weights) in one call, which
+    runs as two launches (82 and 46 levels), every level's input the previous
+    level's output. Sampled outputs (every 256-row slab edge, both ends, random
+    rows) of levels at the start, on both sides of the launch boundary and at
+    the end, against the oracle on the input each level read."""
+    import synthetic
+    dev = torch.device("cuda")
+    layers = []
+    for layer in range(synthetic.LLAMA7B_LAYERS):
+        mats = []
+        for idx, (K, N) in enumerate(synthetic.LLAMA7B_LAYER):
+            W = synthetic.weights(N, K, seed=5000 + 16 * layer + idx, device=dev)
+            mats.append(bl.bin_pack(W, bl.BL_PACK_FBI))
+            del W
+        layers.append(mats)
+    cur = synthetic.activations(M, 4096, seed=77, device=dev)
+    levels = []
+    for mats in layers:
+        q, k, v, o, h = (torch.empty((M, 4096), dtype=torch.bfloat16, device=dev) for _ in range(5))
+        g, u = (torch.empty((M, 11008), dtype=torch.bfloat16, device=dev) for _ in range(2))
+        levels.append((cur, [(mats[0][0], mats[0][1], q), (mats[1][0], mats[1][1], k), (mats[2][0], mats[2][1], v)]))
+        levels.append((v, [(mats[3][0], mats[3][1], o)]))
+        levels.append((o, [(mats[4][0], mats[4][1], g), (mats[5][0], mats[5][1], u)]))
+        levels.append((u, [(mats[6][0], mats[6][1], h)]))
+        cur = h
+    bl.W1A16Stack(levels).run()
+    torch.cuda.synchronize()
+    assert bl.device_error() == (0, 0)
+    for li in (0, 1, 2, 3, 80, 81, 82, 83, 126, 127):
+        xin, lins = levels[li]
+        K = xin.shape[-1]
+        xb = synthetic.bf16_bits(xin.reshape(M, K))
+        for i, (p, a, y) in enumerate(lins):
+            N = p.shape[0]
+            ms, js = sample_positions(M, N, 48, seed=1000 * M + 10 * li + i, tile_m=16, tile_n=256)
+            pk, al = p.cpu().numpy().view(np.uint32), a.cpu().numpy()
+            y_ref = oracle.w1a16_at(xb, pk, al, K, ms, js)
+            y_gpu = bf16_to_f64(y.reshape(M, N))[ms, js]
+            check_w1a16(y_gpu, y_ref, al, xb, ms, js, what=f"level {li} linear {i} (K={K}, N={N})")
 
 
 def test_stack_longer_than_one_launch(bl, oracle):
